@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV decode layer-step on B200.
+
+One step = pa_reshape_and_cache of the step's new token per sequence, then
+pa_decode (partition kernel + partition-merge kernel) over every sequence's
+whole context.  Default workload: the Llama-3-70B GQA decode layer (128
+sequences, 64 q / 8 kv heads, head_dim 128, bf16, 16-token blocks, context
+lengths lognormal with median 2048 clipped to [16, 8192], shuffled pool).
+
+Prints ONE JSON line (rank 0).  `value` = decode algorithmic bytes (K and V
+of every valid context token + q + out) per second, summed over ranks, with
+inputs resident in HBM; the KV pool (~1.2 GB) is far larger than the 126 MB
+L2, so no flush is needed between steps.  Multi-GPU runs are independent
+replicas (weak scaling; decode needs no exchange between GPUs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention HBM GB/s (% of B200 peak); seqs/s per layer-step"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; replicas only)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def reduce_over_ranks(x: float, op: str, world: int, device=None) -> float:
+    """Max or sum of a scalar over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# measured peaks and clocks
+# ---------------------------------------------------------------------------
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", gpu_id], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 8:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[4 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+def describe(spec, ctx, num_blocks):
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    return (f"{spec.name}: {spec.num_seqs} seqs, {spec.n_q_heads} q / {spec.n_kv_heads} kv "
+            f"heads, head_dim {spec.head_dim}, q {W.DTYPE_NAMES[spec.q_dtype]}, kv "
+            f"{W.DTYPE_NAMES[spec.kv_dtype]}, block 16, ctx {spec.ctx_kind}{spec.ctx_args} "
+            f"(sum {int(ctx.sum())} tokens), shuffled pool of {num_blocks} blocks")
+
+
+def get_spec(name):
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    return {"llama3_70b_gqa_bf16": W.LLAMA3_70B_GQA_BF16, "llama2_7b_fp16": W.LLAMA2_7B_FP16,
+            "mixed_step_fp8_decode": W.MIXED_DECODE_FP8, "tiny_fp32": W.TINY_FP32}[name]
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(inp, budget_s: float, max_units=None):
+    """Time the oracle on a bounded prefix of the workload's sequences.
+    Returns (seconds, bytes, seqs, tokens, threads)."""
+    import oracle as orc
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    spec = inp.spec
+    q = inp.q.cpu()
+    bt = inp.block_tables.cpu().numpy()
+    cl = inp.context_lens.cpu().numpy()
+    kp, vp = inp.k_pool, inp.v_pool
+    threads = os.cpu_count() or 1
+    done_s, done_bytes, done_seqs, done_tok = 0.0, 0, 0, 0
+    s = 0
+    chunk = max(1, threads // max(1, spec.n_kv_heads) or 1)
+    while s < spec.num_seqs and done_s < budget_s:
+        idx = list(range(s, min(s + chunk, spec.num_seqs)))
+        need = sorted({int(b) for i in idx for b in bt[i, :-(-int(cl[i]) // 16)]})
+        remap = {b: j for j, b in enumerate(need)}
+        bt2 = np.full((len(idx), bt.shape[1]), -1, np.int32)
+        for r, i in enumerate(idx):
+            n = -(-int(cl[i]) // 16)
+            bt2[r, :n] = [remap[int(b)] for b in bt[i, :n]]
+        import torch
+        sel = torch.tensor(need, dtype=torch.long, device=kp.device)
+        k_sub = kp[sel].cpu() if len(need) else kp[:1].cpu()
+        v_sub = vp[sel].cpu() if len(need) else vp[:1].cpu()
+        t0 = time.perf_counter()
+        orc.paged_decode(q[idx], k_sub, v_sub, bt2, cl[idx], inp.scale, spec.q_dtype,
+                         spec.kv_dtype, inp.k_scale, inp.v_scale, nthreads=threads)
+        done_s += time.perf_counter() - t0
+        done_bytes += W.decode_algorithmic_bytes(cl[idx], spec.n_q_heads, spec.n_kv_heads,
+                                                 spec.head_dim, W.ELEM_BYTES[spec.q_dtype],
+                                                 W.ELEM_BYTES[spec.kv_dtype])
+        done_seqs += len(idx)
+        done_tok += int(cl[idx].sum())
+        s += len(idx)
+    return done_s, done_bytes, done_seqs, done_tok, threads
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local):
+    import torch
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_init(world, "nccl")
+    spec = get_spec(args.workload)
+    inp = W.make_decode_inputs(spec, device=dev)
+    ctx = inp.context_lens.cpu().numpy()
+    n = spec.num_seqs
+    # the step's new token (position ctx-1) of every sequence
+    key, val = W.make_new_kv(n, spec.n_kv_heads, spec.head_dim,
+                             spec.q_dtype if spec.kv_dtype == W.FP8_E4M3 else spec.kv_dtype,
+                             dev, seed=spec.seed + 7)
+    slots = torch.from_numpy(W.slots_from_positions(
+        inp.block_tables.cpu().numpy(), np.arange(n), np.maximum(ctx - 1, 0))).to(dev)
+    slots[torch.from_numpy(ctx == 0).to(dev)] = -1
+    out = torch.empty_like(inp.q)
+    mb = inp.block_tables.shape[1]
+    ws = B.alloc_decode_workspace(inp.q, mb)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    kvdt = B.dtype_code(inp.k_pool)
+    algo_bytes = W.decode_algorithmic_bytes(ctx, spec.n_q_heads, spec.n_kv_heads, spec.head_dim,
+                                            W.ELEM_BYTES[spec.q_dtype], W.ELEM_BYTES[spec.kv_dtype])
+    n_parts = -(-mb * 16 // 512)
+    launches_per_step = 2 + (1 if n_parts > 1 else 0)
+
+    def step(ev_a=None, ev_b=None):
+        B.pa_reshape_and_cache(inp.k_pool, inp.v_pool, key, val, slots, inp.k_scale,
+                               inp.v_scale, dev_err=err)
+        if ev_a is not None:
+            ev_a.record()
+        B.pa_decode_partitions(out, inp.q, inp.k_pool, inp.v_pool, inp.block_tables,
+                               inp.context_lens, inp.scale, inp.k_scale, inp.v_scale,
+                               workspace=ws, dev_err=err)
+        if ev_b is not None:
+            ev_b.record()
+        B.pa_decode_reduce(out, inp.context_lens, mb, kvdt, inp.v_scale, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    time.sleep(0.3)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    t_start.record()
+    for i in range(K):
+        step(*evs[i])
+    t_stop.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clocks = sampler.stop()
+    ms_total = t_start.elapsed_time(t_stop)
+    kern_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_max = reduce_over_ranks(ms_total, "max", world, dev)
+    total_bytes = reduce_over_ranks(algo_bytes * K, "sum", world, dev)
+    value = total_bytes / (ms_max / 1e3) / 1e9
+
+    # ---- end to end through the public API from pinned host buffers
+    q_h = inp.q.cpu().pin_memory()
+    key_h, val_h = key.cpu().pin_memory(), val.cpu().pin_memory()
+    slots_h = slots.cpu().pin_memory()
+    bt_h = inp.block_tables.cpu().pin_memory()
+    cl_h = inp.context_lens.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d, key_d, val_d = torch.empty_like(inp.q), torch.empty_like(key), torch.empty_like(val)
+    slots_d, bt_d, cl_d = torch.empty_like(slots), torch.empty_like(inp.block_tables), \
+        torch.empty_like(inp.context_lens)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, key_h, val_h, slots_h, bt_h, cl_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        for dst, src in ((q_d, q_h), (key_d, key_h), (val_d, val_h), (slots_d, slots_h),
+                         (bt_d, bt_h), (cl_d, cl_h)):
+            dst.copy_(src, non_blocking=True)
+        B.pa_reshape_and_cache(inp.k_pool, inp.v_pool, key_d, val_d, slots_d, inp.k_scale,
+                               inp.v_scale, dev_err=err)
+        B.pa_decode(out, q_d, inp.k_pool, inp.v_pool, bt_d, cl_d, inp.scale, inp.k_scale,
+                    inp.v_scale, workspace=ws, dev_err=err)
+        out_h.copy_(out, non_blocking=True)
+
+    K2 = max(3, min(K, 200))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K2):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e2e_ms = reduce_over_ranks(e0.elapsed_time(e1), "max", world, dev)
+    e2e_value = reduce_over_ranks(algo_bytes * K2, "sum", world, dev) / (e2e_ms / 1e3) / 1e9
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+
+    # ---- roofline of the dominant kernel (partition kernel), live events
+    kern_avg_ms = sum(kern_ms) / len(kern_ms)
+    peak, peak_src = hbm_peak()
+    achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic_from_profile(args.workload),
+                "kernel": "decode_mma_kernel (partition kernel)",
+                "kernel_avg_us": round(kern_avg_ms * 1e3, 2),
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_src == "measured" else "fallback 6.65 TB/s"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype":
+            {W.F32: "f32", W.F16: "f16", W.BF16: "bf16"}[spec.q_dtype]
+            + ("+fp8kv" if spec.kv_dtype == W.FP8_E4M3 else ""),
+        "data": "synthetic (seeded N(0,1) values, seeded context lengths and block shuffle)",
+        "config": {"workload": describe(spec, ctx, inp.num_blocks), "global_batch": n * world,
+                   "seq_len": int(ctx.max()), "tokens_per_step": int(ctx.sum()),
+                   "algorithmic_bytes_per_step": int(algo_bytes),
+                   "step": "reshape_and_cache (1 new token/seq) + decode partitions + reduce",
+                   "l2": "inputs larger than L2 (KV pool > 1 GB vs 126 MB L2); no flush",
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "seqs_per_s": round(n * world / (ms_max / K / 1e3), 1),
+        "tokens_per_s": round(float(ctx.sum()) * world / (ms_max / K / 1e3), 1),
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": K2,
+                "ms_per_step": round(e2e_ms / K2, 4)},
+        "roofline": roofline,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, b, ns, nt, th = oracle_sample(inp, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(b / secs / 1e9, 4), "unit": "GB/s", "cores": th,
+                                "kind": "oracle",
+                                "sample": f"first {ns} of {n} sequences ({nt} tokens) of the "
+                                          f"same workload, {secs:.1f} s, fp64 C oracle"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def traffic_from_profile(workload):
+    """DRAM bytes per launch of the partition kernel from the committed ncu
+    summary, if that summary matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "pagedattention_paged_kv_pa_b200", "csrc", "decode.cu")
+        import hashlib
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if rec.get("decode_cu_sha256_16") != h:
+            return None
+        return rec.get("traffic_bytes_per_launch", {}).get(workload)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle, as it stands
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world, local):
+    if rank != 0:
+        return
+    import torch
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    spec = get_spec(args.workload)
+    inp = W.make_decode_inputs(spec, device="cpu")
+    steps, warm = args.steps, args.warmup
+    per_step = max(0.05, min(2.0, 150.0 / max(1, steps + warm)))
+    for _ in range(warm):
+        oracle_sample(inp, per_step)
+    tot_s = tot_b = 0.0
+    ns = nt = 0
+    th = 1
+    for _ in range(steps):
+        s, b, a, t, th = oracle_sample(inp, per_step)
+        tot_s += s
+        tot_b += b
+        ns, nt = a, t
+    value = tot_b / tot_s / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": steps, "warmup": warm,
+            "ms_per_step": round(1e3 * tot_s / steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(spec, inp.context_lens.numpy(), inp.num_blocks)},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": th,
+                             "kind": "oracle",
+                             "sample": f"each step: first {ns} sequences ({nt} tokens), "
+                                       f"about {per_step:.2f} s of fp64 C oracle work"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_70b_gqa_bf16")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world, local)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,274 @@
+/*
+ * pa.h -- C ABI of the paged-KV attention library (libpa_b200.so, sm_100a).
+ *
+ * The operations follow three web pages on PagedAttention:
+ *  [P1] "LLM inference optimization: KV cache & PagedAttention"
+ *       (carlstack.gravito.dev)
+ *  [P2] "vLLM explained" (jackchen890311.github.io)
+ *  [P3] "Daily AI, 2026-07-31: inference serving" (k1-blog.pages.dev)
+ *
+ * Common conventions
+ * ------------------
+ *  - Pools.  k_pool and v_pool are separate device arrays laid out
+ *    [num_blocks][n_kv_heads][block_size][head_dim] ("HND"): one physical block
+ *    holds the 16 tokens of every KV head ([P2] "Block 的大小怎麼決定": a block
+ *    spans all KV heads), and the 16 x head_dim tile of one (block, head) is
+ *    contiguous.  block_size must be 16 ([P1] §三.1, [P2] "PagedAttention").
+ *  - Block tables.  int32 [num_seqs][max_blocks_per_seq], row-major; entry j of
+ *    a row is the physical block holding logical block j (tokens 16j..16j+15)
+ *    of that sequence ([P1] §三.1 "Logical Block Table"; [P2] "PagedAttention",
+ *    item 3).  Only the first ceil(context_len / 16) entries of a row are read.
+ *  - Slots.  slot = physical_block * 16 + offset; a negative slot means "no
+ *    slot" and is skipped.
+ *  - GQA.  q head h reads kv head h / (n_q_heads / n_kv_heads) ([P2] "Block 的
+ *    大小怎麼決定": GQA/MQA models have fewer KV heads).
+ *  - Ownership.  Every pointer argument is owned by the caller.  Device
+ *    pointers must stay valid until the work queued on `stream` has finished.
+ *    The library allocates no device memory and never synchronises with the
+ *    device on these paths; all work is queued on `stream` (a cudaStream_t;
+ *    NULL means the legacy default stream).
+ *  - Errors.  Argument errors are detected on the host before anything is
+ *    launched and return PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED.  A failed
+ *    launch returns PA_ERR_CUDA.  Data-dependent faults that only the device
+ *    can see (a block id outside [0, num_blocks), a slot outside the pool) are
+ *    never trapped: the offending element is skipped and, when `dev_err` is
+ *    non-NULL, bits of PA_DEVERR_* are OR-ed into *dev_err (a device int32 the
+ *    caller zeroes).  Bounded waits inside kernels that give up set
+ *    PA_DEVERR_TIMEOUT instead of hanging.
+ *  - Thread safety.  The kernels' entry points may be called from several host
+ *    threads.  A pa_alloc handle must not be used by two threads at once.
+ */
+#ifndef PA_B200_H
+#define PA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_ABI_VERSION 1
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,
+    PA_ERR_UNSUPPORTED = 2,
+    PA_ERR_OOM = 3,
+    PA_ERR_CUDA = 4
+} pa_status;
+
+typedef enum {
+    PA_F32 = 0,
+    PA_F16 = 1,
+    PA_BF16 = 2,
+    PA_FP8_E4M3 = 3 /* OCP E4M3FN; stored value x per-tensor scale */
+} pa_dtype;
+
+/* bits OR-ed into *dev_err */
+#define PA_DEVERR_BLOCK_ID 1  /* a block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 2      /* a slot or block-pair id outside the pool */
+#define PA_DEVERR_TIMEOUT 4   /* a bounded wait inside a kernel gave up */
+#define PA_DEVERR_QUERY_LOC 8 /* inconsistent query_start_loc / context_lens */
+
+int pa_abi_version(void);
+const char* pa_status_string(pa_status s);
+
+/* ------------------------------------------------------------------------- */
+/* Decode attention                                                           */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * pa_decode -- one new query token per running sequence attends to that
+ * sequence's whole cached context through its block table:
+ *     out[s][h] = softmax(scale * q[s][h] . K_s^T) . V_s
+ * ([P1] §二 Attention formula; [P1] §一.2: decode re-reads the whole KV cache
+ * every step; [P2] "兩層實作": the kernel reads K/V by jumping through the
+ * block table, and paging leaves the result equal to ordinary attention).
+ * K_s / V_s are the first context_lens[s] tokens of sequence s; context_lens
+ * includes the current token, whose K/V pa_reshape_and_cache wrote earlier in
+ * the step.  A sequence with context 0 gets an all-zero output row.
+ *
+ *   out          device [num_seqs][n_q_heads][head_dim], dtype q_dtype
+ *   q            device [num_seqs][n_q_heads][head_dim], dtype q_dtype
+ *   k_pool/v_pool device pools (see conventions), dtype kv_dtype
+ *   block_tables device int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens device int32 [num_seqs], each in [0, 16 * max_blocks_per_seq]
+ *   scale        multiplies q . k (usually 1/sqrt(head_dim))
+ *   k_scale, v_scale  per-tensor dequantisation scales, used only when
+ *                kv_dtype is PA_FP8_E4M3 (an element's value is code x scale)
+ *   workspace    device scratch of at least pa_decode_workspace_size(...)
+ *                bytes, 16-byte aligned; contents need no initialisation
+ *   dev_err      optional device int32 for PA_DEVERR_* bits
+ *
+ * Supported: block_size 16; head_dim 64 or 128; n_q_heads % n_kv_heads == 0
+ * with group size n_q_heads / n_kv_heads <= 8; (q_dtype, kv_dtype) in
+ * {(F32,F32), (F16,F16), (BF16,BF16), (F16,FP8_E4M3), (BF16,FP8_E4M3)}.
+ * Pointers must be 16-byte aligned.  Output rows are bit-identical under any
+ * permutation of the physical blocks (partitioning and reduction order depend
+ * only on logical positions).
+ *
+ * The work is split along the context into fixed partitions: a partition
+ * kernel writes per-partition (max, sum, unnormalised output) into the
+ * workspace and a reduce kernel merges the partitions of sequences that have
+ * more than one.  pa_decode queues both; pa_decode_partitions and
+ * pa_decode_reduce queue them one at a time (same arguments, same result).
+ */
+size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim,
+                                int max_blocks_per_seq);
+
+pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    int block_size, int n_q_heads, int n_kv_heads, int head_dim,
+                    int num_seqs, int max_blocks_per_seq, int num_blocks,
+                    pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
+                    void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                    void* stream);
+
+pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool,
+                               const void* v_pool, const int32_t* block_tables,
+                               const int32_t* context_lens, float scale, int block_size,
+                               int n_q_heads, int n_kv_heads, int head_dim, int num_seqs,
+                               int max_blocks_per_seq, int num_blocks, pa_dtype q_dtype,
+                               pa_dtype kv_dtype, float k_scale, float v_scale,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                               void* stream);
+
+pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads,
+                           int head_dim, int num_seqs, int max_blocks_per_seq,
+                           pa_dtype q_dtype, pa_dtype kv_dtype, float v_scale,
+                           const void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Chunked prefill                                                            */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * pa_prefill_paged -- chunked prefill: a long prompt is cut into chunks that
+ * are batched with decodes ([P1] §六.2 "Chunked Prefill"; [P2] "附錄與延伸").
+ * Chunk c owns query rows query_start_loc[c] .. query_start_loc[c+1]-1 (L_c
+ * rows) and its sequence holds context_lens[c] tokens including the chunk, so
+ * its history is H_c = context_lens[c] - L_c.  The chunk's K/V must already be
+ * in the pools (pa_reshape_and_cache).  Query i of the chunk sits at absolute
+ * position H_c + i and attends causally to keys 0 .. H_c + i:
+ *     out[r][h] = softmax(scale * q[r][h] . K^T, masked) . V
+ * The prefill half of a batch is compute-bound ([P1] §一.1; [P3] "prefill 與
+ * decode"); this kernel runs the two contractions on tcgen05 tensor cores.
+ *
+ *   out, q         device [total_q][n_q_heads][head_dim], dtype q_dtype,
+ *                  total_q = query_start_loc[n_chunks]
+ *   block_tables   device int32 [n_chunks][max_blocks_per_seq]
+ *   query_start_loc device int32 [n_chunks + 1], non-decreasing, [0] = 0
+ *   context_lens   device int32 [n_chunks], context_lens[c] >= L_c
+ *   max_chunk_len  host bound on every L_c (sizes the grid; no device sync)
+ *
+ * Supported: block_size 16, head_dim 128, group size <= 8, q_dtype BF16 and
+ * kv_dtype BF16 or FP8_E4M3 (FP8 K/V are widened to bf16 in shared memory,
+ * exactly).  The output is written in q_dtype.
+ */
+pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
+                           const int32_t* block_tables, const int32_t* query_start_loc,
+                           const int32_t* context_lens, float scale, int block_size,
+                           int n_q_heads, int n_kv_heads, int head_dim, int n_chunks,
+                           int max_chunk_len, int max_blocks_per_seq, int num_blocks,
+                           pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale,
+                           float v_scale, int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Slot write and copy-on-write block copy                                    */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V rows into the slot
+ * its position maps to (the block table gives the block, the position modulo
+ * 16 the offset; [P2] "PagedAttention" items 1-4, [P1] §三.1).
+ *
+ *   key, value   device [num_tokens][n_kv_heads][head_dim], dtype src_dtype
+ *   slot_mapping device int64 [num_tokens]; < 0 skips the token; slots must be
+ *                distinct (two tokens writing one slot race)
+ *   cache_dtype  == src_dtype: bytes are copied;
+ *                PA_FP8_E4M3 (src F16/BF16/F32): code = RNE_satfinite(x / scale)
+ *                with the quotient taken in binary32, k_scale for K and
+ *                v_scale for V ([P2] "Block 的大小怎麼決定": FP8 is 1 byte).
+ * Out-of-range slots are skipped and flagged with PA_DEVERR_SLOT.
+ */
+pa_status pa_reshape_and_cache(void* k_pool, void* v_pool, const void* key, const void* value,
+                               const int64_t* slot_mapping, int num_tokens, int n_kv_heads,
+                               int head_dim, int block_size, int num_blocks,
+                               pa_dtype src_dtype, pa_dtype cache_dtype, float k_scale,
+                               float v_scale, int32_t* dev_err, void* stream);
+
+/*
+ * pa_copy_blocks -- the copy half of copy-on-write: when a branch is about to
+ * write into a block it shares, the block is first copied to a private one
+ * ([P1] §三.2; [P2] "帶來的好處").  For each pair (src, dst) the whole dst
+ * block (every KV head, K and V) becomes a byte copy of the src block.
+ *
+ *   block_pairs  device int64 [n_pairs][2] = (src, dst); dst ids must be
+ *                distinct and must not appear as a src (pa_alloc_prepare_write
+ *                produces such pairs).  Ids outside [0, num_blocks) are skipped
+ *                and flagged with PA_DEVERR_SLOT.
+ */
+pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_pairs, int n_pairs,
+                         int n_kv_heads, int head_dim, int block_size, int num_blocks,
+                         pa_dtype kv_dtype, int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Host block allocator (not on the hot path)                                 */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * The memory-management layer: fixed-size blocks, a block table per
+ * sequence, allocation on demand, release when a request finishes
+ * ([P2] "PagedAttention" items 1-4, "兩層實作"), sharing by reference count and
+ * copy-on-write ([P1] §三.2), and a block in use is never handed out again
+ * ([P2] "KV cache 什麼時候可以被覆蓋").
+ *
+ * Free blocks are handed out FIFO from `initial_free_order` (NULL: 0..N-1;
+ * otherwise a permutation of 0..N-1) and freed blocks join the back of the
+ * queue, so the state after any call sequence is deterministic.  Every call is
+ * all-or-nothing: PA_ERR_OOM or PA_ERR_INVALID_ARG leave the state unchanged.
+ * Sequence ids are arbitrary int64 values.  Handles are not thread-safe.
+ */
+typedef struct pa_alloc pa_alloc;
+
+/* NULL on invalid arguments (num_blocks < 1, block_size != 16, bad order) */
+pa_alloc* pa_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_order);
+void pa_alloc_destroy(pa_alloc* a);
+
+/* Reserve slots for n_tokens new tokens of `seq` (created on first use),
+ * taking new blocks when the last one is full.  slots_out[n_tokens] receives
+ * their slots (may be NULL when n_tokens == 0).  Refused with
+ * PA_ERR_INVALID_ARG while the last block is partially filled and shared:
+ * call pa_alloc_prepare_write first. */
+pa_status pa_alloc_append(pa_alloc* a, int64_t seq, int n_tokens, int64_t* slots_out);
+
+/* `child` (new id) gets the parent's table; every block's count goes up by 1. */
+pa_status pa_alloc_fork(pa_alloc* a, int64_t parent, int64_t child);
+
+/* If the last block of `seq` is partially filled and shared, move `seq` to a
+ * fresh block and report the pair (old, new) that pa_copy_blocks must copy
+ * before the next write; cow_pairs_out has room for one pair (2 int64).
+ * *n_pairs_out is 0 or 1. */
+pa_status pa_alloc_prepare_write(pa_alloc* a, int64_t seq, int64_t* cow_pairs_out,
+                                 int* n_pairs_out);
+
+/* Drop `seq`; each of its blocks' counts goes down by 1 and a block whose
+ * count reaches 0 joins the back of the free queue (in logical order). */
+pa_status pa_alloc_free_seq(pa_alloc* a, int64_t seq);
+
+/* Copy the block table of `seq` (logical order) into out[cap]; *n_out gets
+ * its length.  PA_ERR_INVALID_ARG if cap is too small or seq is unknown. */
+pa_status pa_alloc_block_table(const pa_alloc* a, int64_t seq, int32_t* out, int cap,
+                               int* n_out);
+/* Copy the free queue (front first) into out[cap]. */
+pa_status pa_alloc_free_list(const pa_alloc* a, int32_t* out, int cap, int* n_out);
+int pa_alloc_num_tokens(const pa_alloc* a, int64_t seq); /* -1 if unknown */
+int pa_alloc_refcount(const pa_alloc* a, int32_t block); /* -1 if out of range */
+int pa_alloc_num_free(const pa_alloc* a);
+int pa_alloc_num_seqs(const pa_alloc* a);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PA_B200_H */

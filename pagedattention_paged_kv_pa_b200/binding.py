@@ -1,0 +1,298 @@
+"""Thin Python binding of libpa_b200.so (the C ABI in include/pa.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  Functions keep the C names and take torch tensors (device
+memory) for the device pointers; shapes and dtypes are read off the tensors,
+the stream is torch's current stream unless one is given.  If the shared
+library is missing this module raises on import -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa_b200.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_OOM, PA_ERR_CUDA = range(5)
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = range(4)
+PA_DEVERR_BLOCK_ID, PA_DEVERR_SLOT, PA_DEVERR_TIMEOUT, PA_DEVERR_QUERY_LOC = 1, 2, 4, 8
+
+# every symbol include/pa.h declares
+EXPORTS = (
+    "pa_abi_version", "pa_status_string", "pa_decode_workspace_size", "pa_decode",
+    "pa_decode_partitions", "pa_decode_reduce", "pa_prefill_paged", "pa_reshape_and_cache",
+    "pa_copy_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_append",
+    "pa_alloc_fork", "pa_alloc_prepare_write", "pa_alloc_free_seq", "pa_alloc_block_table",
+    "pa_alloc_free_list", "pa_alloc_num_tokens", "pa_alloc_refcount", "pa_alloc_num_free",
+    "pa_alloc_num_seqs",
+)
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m pagedattention_paged_kv_pa_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_int64
+    L.pa_abi_version.restype = I
+    L.pa_status_string.argtypes = [I]
+    L.pa_status_string.restype = ctypes.c_char_p
+    L.pa_decode_workspace_size.argtypes = [I, I, I, I]
+    L.pa_decode_workspace_size.restype = Z
+    dec = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, F, F, P, Z, P, P]
+    L.pa_decode.argtypes = dec
+    L.pa_decode_partitions.argtypes = dec
+    L.pa_decode_reduce.argtypes = [P, P, I, I, I, I, I, I, F, P, Z, P]
+    L.pa_prefill_paged.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, F, F,
+                                   P, P]
+    L.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, F, P, P]
+    L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
+    for fn in ("pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_prefill_paged",
+               "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_append", "pa_alloc_fork",
+               "pa_alloc_prepare_write", "pa_alloc_free_seq", "pa_alloc_block_table",
+               "pa_alloc_free_list"):
+        getattr(L, fn).restype = I
+    L.pa_alloc_create.argtypes = [I, I, P]
+    L.pa_alloc_create.restype = P
+    L.pa_alloc_destroy.argtypes = [P]
+    L.pa_alloc_destroy.restype = None
+    L.pa_alloc_append.argtypes = [P, I64, I, P]
+    L.pa_alloc_fork.argtypes = [P, I64, I64]
+    L.pa_alloc_prepare_write.argtypes = [P, I64, P, P]
+    L.pa_alloc_free_seq.argtypes = [P, I64]
+    L.pa_alloc_block_table.argtypes = [P, I64, P, I, P]
+    L.pa_alloc_free_list.argtypes = [P, P, I, P]
+    L.pa_alloc_num_tokens.argtypes = [P, I64]
+    L.pa_alloc_refcount.argtypes = [P, ctypes.c_int32]
+    L.pa_alloc_num_free.argtypes = [P]
+    L.pa_alloc_num_seqs.argtypes = [P]
+    for fn in ("pa_alloc_num_tokens", "pa_alloc_refcount", "pa_alloc_num_free",
+               "pa_alloc_num_seqs"):
+        getattr(L, fn).restype = I
+    return L
+
+
+lib = _load()
+
+_DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
+       torch.uint8: PA_FP8_E4M3, torch.float8_e4m3fn: PA_FP8_E4M3}
+
+
+def status_string(s: int) -> str:
+    return lib.pa_status_string(s).decode()
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise PAError(PA_ERR_UNSUPPORTED, f"dtype {t.dtype}") from None
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, what: str):
+    if status != PA_OK:
+        raise PAError(status, what)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise PAError(PA_ERR_INVALID_ARG, "tensors must be contiguous")
+
+
+# --------------------------------------------------------------------------
+# decode
+# --------------------------------------------------------------------------
+
+def pa_decode_workspace_size(num_seqs: int, n_q_heads: int, head_dim: int,
+                             max_blocks_per_seq: int) -> int:
+    return lib.pa_decode_workspace_size(num_seqs, n_q_heads, head_dim, max_blocks_per_seq)
+
+
+def alloc_decode_workspace(q: torch.Tensor, max_blocks_per_seq: int) -> torch.Tensor:
+    n = pa_decode_workspace_size(q.shape[0], q.shape[1], q.shape[2], max_blocks_per_seq)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+
+
+def _decode_args(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale, v_scale,
+                 workspace, dev_err, stream):
+    _contig(out, q, k_pool, v_pool, block_tables, context_lens)
+    num_seqs, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_pool.shape
+    if d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != tuple(q.shape):
+        raise PAError(PA_ERR_INVALID_ARG, "pa_decode shapes")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PAError(PA_ERR_INVALID_ARG, "block_tables / context_lens must be int32")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return (_p(out), _p(q), _p(k_pool), _p(v_pool), _p(block_tables), _p(context_lens),
+            float(scale), bs, n_q, n_kv, d, num_seqs, block_tables.shape[1], num_blocks,
+            dtype_code(q), dtype_code(k_pool), float(k_scale), float(v_scale), _p(workspace),
+            ws_bytes, _p(dev_err), _stream(stream, q.device))
+
+
+def pa_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale=1.0,
+              v_scale=1.0, workspace=None, dev_err=None, stream=None):
+    """out[s][h] = softmax(scale * q[s][h] . K^T) V over the paged cache."""
+    if workspace is None:
+        workspace = alloc_decode_workspace(q, block_tables.shape[1])
+    _check(lib.pa_decode(*_decode_args(out, q, k_pool, v_pool, block_tables, context_lens,
+                                       scale, k_scale, v_scale, workspace, dev_err, stream)),
+           "pa_decode")
+    return out
+
+
+def pa_decode_partitions(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                         k_scale=1.0, v_scale=1.0, workspace=None, dev_err=None, stream=None):
+    _check(lib.pa_decode_partitions(*_decode_args(out, q, k_pool, v_pool, block_tables,
+                                                  context_lens, scale, k_scale, v_scale,
+                                                  workspace, dev_err, stream)),
+           "pa_decode_partitions")
+
+
+def pa_decode_reduce(out, context_lens, max_blocks_per_seq, kv_dtype, v_scale=1.0,
+                     workspace=None, stream=None):
+    num_seqs, n_q, d = out.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_reduce(_p(out), _p(context_lens), n_q, d, num_seqs, max_blocks_per_seq,
+                                dtype_code(out), kv_dtype, float(v_scale), _p(workspace),
+                                ws_bytes, _stream(stream, out.device)), "pa_decode_reduce")
+
+
+# --------------------------------------------------------------------------
+# prefill
+# --------------------------------------------------------------------------
+
+def pa_prefill_paged(out, q, k_pool, v_pool, block_tables, query_start_loc, context_lens,
+                     scale, max_chunk_len, k_scale=1.0, v_scale=1.0, dev_err=None,
+                     stream=None):
+    _contig(out, q, k_pool, v_pool, block_tables, query_start_loc, context_lens)
+    total_q, n_q, d = q.shape
+    num_blocks, n_kv, bs, _ = k_pool.shape
+    _check(lib.pa_prefill_paged(_p(out), _p(q), _p(k_pool), _p(v_pool), _p(block_tables),
+                                _p(query_start_loc), _p(context_lens), float(scale), bs, n_q,
+                                n_kv, d, context_lens.shape[0], int(max_chunk_len),
+                                block_tables.shape[1], num_blocks, dtype_code(q),
+                                dtype_code(k_pool), float(k_scale), float(v_scale),
+                                _p(dev_err), _stream(stream, q.device)), "pa_prefill_paged")
+    return out
+
+
+# --------------------------------------------------------------------------
+# slot write / block copy
+# --------------------------------------------------------------------------
+
+def pa_reshape_and_cache(k_pool, v_pool, key, value, slot_mapping, k_scale=1.0, v_scale=1.0,
+                         dev_err=None, stream=None):
+    _contig(k_pool, v_pool, key, value, slot_mapping)
+    if slot_mapping.dtype != torch.int64:
+        raise PAError(PA_ERR_INVALID_ARG, "slot_mapping must be int64")
+    num_tokens, n_kv, d = key.shape
+    num_blocks, _, bs, _ = k_pool.shape
+    _check(lib.pa_reshape_and_cache(_p(k_pool), _p(v_pool), _p(key), _p(value),
+                                    _p(slot_mapping), num_tokens, n_kv, d, bs, num_blocks,
+                                    dtype_code(key), dtype_code(k_pool), float(k_scale),
+                                    float(v_scale), _p(dev_err), _stream(stream, key.device)),
+           "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_pool, v_pool, block_pairs, dev_err=None, stream=None):
+    _contig(k_pool, v_pool, block_pairs)
+    if block_pairs.dtype != torch.int64:
+        raise PAError(PA_ERR_INVALID_ARG, "block_pairs must be int64 [n][2]")
+    num_blocks, n_kv, bs, d = k_pool.shape
+    n_pairs = block_pairs.numel() // 2
+    _check(lib.pa_copy_blocks(_p(k_pool), _p(v_pool), _p(block_pairs), n_pairs, n_kv, d, bs,
+                              num_blocks, dtype_code(k_pool), _p(dev_err),
+                              _stream(stream, k_pool.device)), "pa_copy_blocks")
+
+
+# --------------------------------------------------------------------------
+# host allocator
+# --------------------------------------------------------------------------
+
+class BlockAllocator:
+    """Owning wrapper of a pa_alloc handle (see include/pa.h)."""
+
+    def __init__(self, num_blocks: int, block_size: int = 16, initial_free_order=None):
+        self.num_blocks = num_blocks
+        self._lib = lib  # kept so __del__ still works during interpreter shutdown
+        order = None
+        if initial_free_order is not None:
+            arr = (ctypes.c_int32 * num_blocks)(*initial_free_order)
+            order = ctypes.cast(arr, ctypes.c_void_p)
+        self._h = lib.pa_alloc_create(num_blocks, block_size, order)
+        if not self._h:
+            raise PAError(PA_ERR_INVALID_ARG, "pa_alloc_create")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            self._lib.pa_alloc_destroy(h)
+            self._h = None
+
+    def append(self, seq: int, n_tokens: int):
+        """Returns (status, slots list)."""
+        buf = (ctypes.c_int64 * max(n_tokens, 1))()
+        st = lib.pa_alloc_append(self._h, seq, n_tokens, ctypes.cast(buf, ctypes.c_void_p))
+        return st, (list(buf[:n_tokens]) if st == PA_OK else [])
+
+    def fork(self, parent: int, child: int) -> int:
+        return lib.pa_alloc_fork(self._h, parent, child)
+
+    def prepare_write(self, seq: int):
+        buf = (ctypes.c_int64 * 2)()
+        n = ctypes.c_int(0)
+        st = lib.pa_alloc_prepare_write(self._h, seq, ctypes.cast(buf, ctypes.c_void_p),
+                                        ctypes.byref(n))
+        return st, ([(buf[0], buf[1])] if (st == PA_OK and n.value == 1) else [])
+
+    def free_seq(self, seq: int) -> int:
+        return lib.pa_alloc_free_seq(self._h, seq)
+
+    def block_table(self, seq: int):
+        cap = self.num_blocks
+        buf = (ctypes.c_int32 * cap)()
+        n = ctypes.c_int(0)
+        st = lib.pa_alloc_block_table(self._h, seq, ctypes.cast(buf, ctypes.c_void_p), cap,
+                                      ctypes.byref(n))
+        _check(st, "pa_alloc_block_table")
+        return list(buf[:n.value])
+
+    def free_list(self):
+        buf = (ctypes.c_int32 * self.num_blocks)()
+        n = ctypes.c_int(0)
+        _check(lib.pa_alloc_free_list(self._h, ctypes.cast(buf, ctypes.c_void_p),
+                                      self.num_blocks, ctypes.byref(n)), "pa_alloc_free_list")
+        return list(buf[:n.value])
+
+    def num_tokens(self, seq: int) -> int:
+        return lib.pa_alloc_num_tokens(self._h, seq)
+
+    def refcount(self, block: int) -> int:
+        return lib.pa_alloc_refcount(self._h, block)
+
+    def num_free(self) -> int:
+        return lib.pa_alloc_num_free(self._h)
+
+    def num_seqs(self) -> int:
+        return lib.pa_alloc_num_seqs(self._h)

@@ -1,0 +1,327 @@
+// C ABI shim: validates arguments on the host, sizes the decode workspace,
+// builds (and caches) TMA tensor maps over the KV pools, and queues the
+// kernels on the caller's stream.  No device memory is allocated here and no
+// call synchronises with the device.
+#include <mutex>
+#include <vector>
+
+#include "pa_internal.h"
+
+namespace {
+
+using pa::DecodeParams;
+using pa::ReduceParams;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(pa_dtype d) {
+  switch (d) {
+    case PA_F32: return 4;
+    case PA_F16: return 2;
+    case PA_BF16: return 2;
+    case PA_FP8_E4M3: return 1;
+  }
+  return 0;
+}
+
+bool valid_dtype(int d) { return d >= PA_F32 && d <= PA_FP8_E4M3; }
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeFn>(nullptr);
+    return reinterpret_cast<EncodeFn>(p);
+  }();
+  return fn;
+}
+
+struct MapKey {
+  const void* ptr;
+  uint64_t rows;
+  uint32_t cols, esize, box_x, box_y, swz;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && esize == o.esize &&
+           box_x == o.box_x && box_y == o.box_y && swz == o.swz;
+  }
+};
+
+struct MapCache {
+  std::mutex mu;
+  std::vector<std::pair<MapKey, CUtensorMap>> entries;  // most recent last
+};
+
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+
+// A 2-D map over a row-major [rows][cols] array of `esize`-byte elements with a
+// (box_x cols) x (box_y rows) box and the given swizzle.  Returns false if the
+// driver refuses it.
+bool get_map(const void* ptr, uint64_t rows, uint32_t cols, uint32_t esize, uint32_t box_x,
+             uint32_t box_y, CUtensorMapSwizzle swz, CUtensorMap* out) {
+  MapKey key{ptr, rows, cols, esize, box_x, box_y, static_cast<uint32_t>(swz)};
+  MapCache& c = map_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  for (size_t i = 0; i < c.entries.size(); ++i)
+    if (c.entries[i].first == key) {
+      *out = c.entries[i].second;
+      return true;
+    }
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMap m;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esize};
+  const cuuint32_t box[2] = {box_x, box_y};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      esize == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  if (fn(&m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  if (c.entries.size() >= 64) c.entries.erase(c.entries.begin());
+  c.entries.emplace_back(key, m);
+  *out = m;
+  return true;
+}
+
+// Map over a KV pool viewed as [num_blocks * n_kv * 16][head_dim]: one box is a
+// 16-token tile (or its first/second 64-column half for 16-bit head_dim 128),
+// written to shared memory with the swizzle the decode kernel reads with.
+bool kv_pool_map(const void* pool, int num_blocks, int n_kv, int d, pa_dtype dt, CUtensorMap* m) {
+  const uint32_t es = elem_bytes(dt);
+  const uint32_t row_bytes = d * es;
+  const uint32_t box_x = row_bytes > 128 ? 128 / es : d;
+  const CUtensorMapSwizzle swz =
+      (box_x * es == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return get_map(pool, (uint64_t)num_blocks * n_kv * 16, d, es, box_x, 16, swz, m);
+}
+
+// ------------------------------------------------------------ decode checks
+
+struct DecodeShape {
+  int n_q, n_kv, d, num_seqs, max_blocks, num_blocks, n_parts;
+};
+
+pa_status check_decode(const DecodeShape& s, int block_size, pa_dtype q_dt, pa_dtype kv_dt) {
+  if (block_size != 16) return PA_ERR_UNSUPPORTED;
+  if (s.d != 64 && s.d != 128) return PA_ERR_UNSUPPORTED;
+  if (s.n_q < 1 || s.n_kv < 1 || s.n_q % s.n_kv != 0) return PA_ERR_INVALID_ARG;
+  if (s.n_q / s.n_kv > 8) return PA_ERR_UNSUPPORTED;
+  if (s.num_seqs < 0 || s.max_blocks < 1 || s.num_blocks < 1) return PA_ERR_INVALID_ARG;
+  if (s.num_seqs > 65535 || s.n_kv > 65535) return PA_ERR_UNSUPPORTED;
+  if ((int64_t)s.num_blocks * s.n_kv * 16 >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+  if ((int64_t)s.max_blocks * 16 >= (int64_t(1) << 30)) return PA_ERR_UNSUPPORTED;
+  if (!valid_dtype(q_dt) || !valid_dtype(kv_dt)) return PA_ERR_INVALID_ARG;
+  const bool ok = (q_dt == PA_F32 && kv_dt == PA_F32) || (q_dt == PA_F16 && kv_dt == PA_F16) ||
+                  (q_dt == PA_BF16 && kv_dt == PA_BF16) ||
+                  ((q_dt == PA_F16 || q_dt == PA_BF16) && kv_dt == PA_FP8_E4M3);
+  return ok ? PA_OK : PA_ERR_UNSUPPORTED;
+}
+
+size_t ws_o_bytes(const DecodeShape& s) {
+  return (size_t)s.num_seqs * s.n_q * s.n_parts * s.d * sizeof(float);
+}
+size_t ws_total_bytes(const DecodeShape& s) {
+  const size_t o = (ws_o_bytes(s) + 255) & ~size_t(255);
+  return o + (size_t)s.num_seqs * s.n_q * s.n_parts * sizeof(float2);
+}
+
+pa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int pa_abi_version(void) { return PA_ABI_VERSION; }
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_OOM: return "out of blocks";
+    case PA_ERR_CUDA: return "CUDA launch failed";
+  }
+  return "unknown status";
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim, int max_blocks_per_seq) {
+  if (num_seqs < 0 || n_q_heads < 1 || head_dim < 1 || max_blocks_per_seq < 1) return 0;
+  DecodeShape s{n_q_heads, 1, head_dim, num_seqs, max_blocks_per_seq, 1,
+                pa::decode_num_parts(max_blocks_per_seq)};
+  if (s.n_parts <= 1) return 0;
+  return ws_total_bytes(s);
+}
+
+pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, const int32_t* context_lens,
+                               float scale, int block_size, int n_q_heads, int n_kv_heads,
+                               int head_dim, int num_seqs, int max_blocks_per_seq,
+                               int num_blocks, pa_dtype q_dtype, pa_dtype kv_dtype,
+                               float k_scale, float v_scale, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  DecodeShape s{n_q_heads, n_kv_heads, head_dim, num_seqs, max_blocks_per_seq, num_blocks,
+                pa::decode_num_parts(max_blocks_per_seq)};
+  pa_status st = check_decode(s, block_size, q_dtype, kv_dtype);
+  if (st != PA_OK) return st;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
+    return PA_ERR_INVALID_ARG;
+  if (!(scale == scale) || (kv_dtype == PA_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)))
+    return PA_ERR_INVALID_ARG;
+  if (s.n_parts > 1) {
+    if (!workspace || !aligned16(workspace) || workspace_bytes < ws_total_bytes(s))
+      return PA_ERR_INVALID_ARG;
+  }
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = workspace ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
+                                                  ((ws_o_bytes(s) + 255) & ~size_t(255)))
+                      : nullptr;
+  p.dev_err = dev_err;
+  p.scale_log2 = scale * kLog2e * (fp8 ? k_scale : 1.f);
+  p.out_mul = fp8 ? v_scale : 1.f;
+  p.n_q = n_q_heads;
+  p.n_kv = n_kv_heads;
+  p.group = n_q_heads / n_kv_heads;
+  p.num_seqs = num_seqs;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.n_parts_max = s.n_parts;
+  CUtensorMap tmk, tmv;
+  if (pa::decode_uses_tma(q_dtype, kv_dtype)) {
+    if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
+        !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv))
+      return PA_ERR_CUDA;
+  }
+  return cuda_status(pa::launch_decode_partitions(p, head_dim, q_dtype, kv_dtype, &tmk, &tmv,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads, int head_dim,
+                           int num_seqs, int max_blocks_per_seq, pa_dtype q_dtype,
+                           pa_dtype kv_dtype, float v_scale, const void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_seqs < 0 || n_q_heads < 1 || max_blocks_per_seq < 1) return PA_ERR_INVALID_ARG;
+  if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype) || q_dtype == PA_FP8_E4M3)
+    return PA_ERR_INVALID_ARG;
+  DecodeShape s{n_q_heads, 1, head_dim, num_seqs, max_blocks_per_seq, 1,
+                pa::decode_num_parts(max_blocks_per_seq)};
+  if (num_seqs == 0 || s.n_parts <= 1) return PA_OK;
+  if (!out || !context_lens || !workspace || !aligned16(out) || !aligned16(workspace) ||
+      workspace_bytes < ws_total_bytes(s))
+    return PA_ERR_INVALID_ARG;
+  ReduceParams r;
+  r.out = out;
+  r.context_lens = context_lens;
+  r.ws_o = static_cast<const float*>(workspace);
+  r.ws_ml = reinterpret_cast<const float2*>(static_cast<const char*>(workspace) +
+                                            ((ws_o_bytes(s) + 255) & ~size_t(255)));
+  r.out_mul = kv_dtype == PA_FP8_E4M3 ? v_scale : 1.f;
+  r.n_q = n_q_heads;
+  r.num_seqs = num_seqs;
+  r.max_blocks = max_blocks_per_seq;
+  r.n_parts_max = s.n_parts;
+  return cuda_status(pa::launch_decode_reduce(r, head_dim, q_dtype,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    int block_size, int n_q_heads, int n_kv_heads, int head_dim, int num_seqs,
+                    int max_blocks_per_seq, int num_blocks, pa_dtype q_dtype, pa_dtype kv_dtype,
+                    float k_scale, float v_scale, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_err, void* stream) {
+  pa_status st = pa_decode_partitions(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                                      block_size, n_q_heads, n_kv_heads, head_dim, num_seqs,
+                                      max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                                      v_scale, workspace, workspace_bytes, dev_err, stream);
+  if (st != PA_OK) return st;
+  return pa_decode_reduce(out, context_lens, n_q_heads, head_dim, num_seqs, max_blocks_per_seq,
+                          q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_reshape_and_cache(void* k_pool, void* v_pool, const void* key, const void* value,
+                               const int64_t* slot_mapping, int num_tokens, int n_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype src_dtype,
+                               pa_dtype cache_dtype, float k_scale, float v_scale,
+                               int32_t* dev_err, void* stream) {
+  if (block_size != 16) return PA_ERR_UNSUPPORTED;
+  if (num_tokens < 0 || n_kv_heads < 1 || head_dim < 1 || num_blocks < 1)
+    return PA_ERR_INVALID_ARG;
+  if (!valid_dtype(src_dtype) || !valid_dtype(cache_dtype) || src_dtype == PA_FP8_E4M3)
+    return PA_ERR_UNSUPPORTED;
+  if (cache_dtype != src_dtype && cache_dtype != PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
+  if ((head_dim * elem_bytes(src_dtype)) % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_pool || !v_pool || !key || !value || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(key) || !aligned16(value))
+    return PA_ERR_INVALID_ARG;
+  if (cache_dtype == PA_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)) return PA_ERR_INVALID_ARG;
+  pa::ScatterParams p;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.key = key;
+  p.value = value;
+  p.slot_mapping = slot_mapping;
+  p.dev_err = dev_err;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.num_tokens = num_tokens;
+  p.n_kv = n_kv_heads;
+  p.head_dim = head_dim;
+  p.num_blocks = num_blocks;
+  return cuda_status(pa::launch_reshape_and_cache(p, src_dtype, cache_dtype,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_pairs, int n_pairs,
+                         int n_kv_heads, int head_dim, int block_size, int num_blocks,
+                         pa_dtype kv_dtype, int32_t* dev_err, void* stream) {
+  if (block_size != 16) return PA_ERR_UNSUPPORTED;
+  if (n_pairs < 0 || n_kv_heads < 1 || head_dim < 1 || num_blocks < 1 || !valid_dtype(kv_dtype))
+    return PA_ERR_INVALID_ARG;
+  if (n_pairs > 65535) return PA_ERR_UNSUPPORTED;
+  const int64_t bb = (int64_t)n_kv_heads * 16 * head_dim * elem_bytes(kv_dtype);
+  if (bb % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (n_pairs == 0) return PA_OK;
+  if (!k_pool || !v_pool || !block_pairs || !aligned16(k_pool) || !aligned16(v_pool))
+    return PA_ERR_INVALID_ARG;
+  pa::CopyParams p;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.pairs = block_pairs;
+  p.dev_err = dev_err;
+  p.n_pairs = n_pairs;
+  p.num_blocks = num_blocks;
+  p.block_bytes = bb;
+  return cuda_status(pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,618 @@
+// Paged decode attention for sm_100a.
+//
+// One new query token per sequence attends to its whole cached context,
+// softmax(scale * q . K^T) . V ("LLM inference optimization: KV cache &
+// PagedAttention", §二), reading K/V block by block through the sequence's
+// block table ("vLLM explained", "兩層實作").  Decode re-reads the whole cache
+// each step and is bound by HBM bandwidth (same page, §一.2), so the design
+// goal is to keep enough bytes in flight and to touch every byte once.
+//
+// Split-context scheme.  Grid = (context partition, kv head, sequence); a
+// partition is kPart = 512 consecutive logical tokens (32 blocks).  Each CTA:
+//   * one producer warp streams the partition's 16-token K and V tiles with
+//     2-D TMA loads (no multicast) into an 8-stage shared-memory ring guarded
+//     by mbarriers -- the block table indirection becomes one TMA row
+//     coordinate per tile;
+//   * four consumer warps take blocks round-robin; each keeps an online
+//     max / sum / output state for all G query heads of the kv head, so every
+//     K/V byte loaded serves the whole GQA group;
+//   * the warps' states are merged in shared memory; a sequence with one
+//     partition is written straight to `out`, otherwise the partition's
+//     (max, sum, unnormalised output) goes to the workspace and the reduce
+//     kernel merges partitions in fixed order.
+// Work assignment depends only on logical positions, so results are the same
+// bits for any permutation of the physical blocks.
+//
+// Per-block math (16-bit and fp8 caches): S^T[16 tok][8 heads] = K . Q^T and
+// O^T[d][8 heads] += V^T . P^T, each as m16n8k16 warp MMAs with the GQA group
+// as N=8 (fp32 accumulate).  For fp8 caches the E4M3 codes are widened to f16
+// exactly (K in registers, V through a per-warp shared tile) and the
+// per-tensor scales are applied to the scores and to the final output.  fp32
+// inputs use a CUDA-core path with fp32 arithmetic throughout.
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kNW = 4;  // consumer warps
+constexpr int kThreads = (kNW + 1) * 32;
+constexpr int kPartBlocks = kPart / 16;
+constexpr int kStages = 8;
+constexpr int kMaxGroup = 8;
+
+template <int D, bool FP8>
+struct MmaLayout {
+  static constexpr int kTileBytes = 16 * D * (FP8 ? 1 : 2);  // one (block, head) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;          // K + V
+  static constexpr int kConvBytes = FP8 ? 16 * D * 2 : 0;     // per-warp f16 V tile
+  static constexpr int kConvOff = kStages * kStageBytes;
+  static constexpr int kIdsOff = kConvOff + kNW * kConvBytes;
+  static constexpr int kBarOff = kIdsOff + kPartBlocks * 4;
+  static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 1024;  // + align slack
+  static constexpr int kMergeFloats = kNW * kMaxGroup * D + 4 * kNW * kMaxGroup + 2 * kMaxGroup;
+  static_assert(kMergeFloats * 4 <= kIdsOff, "merge scratch must fit in the ring");
+  static_assert(kStageBytes % 1024 == 0 && kConvBytes % 1024 == 0, "1024-B aligned tiles");
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+
+// Clamp a context length into [0, capacity]; a length beyond the table's
+// capacity is a caller error that is flagged, never read past.
+__device__ __forceinline__ int clamp_ctx(int ctx, int cap, int32_t* dev_err, bool report) {
+  if (ctx > cap) {
+    if (report) flag_error(dev_err, PA_DEVERR_BLOCK_ID);
+    return cap;
+  }
+  return ctx < 0 ? 0 : ctx;
+}
+
+// Merge the consumer warps' (m, l, O) states held in shared memory and write
+// the partition result.  mo: [kNW][8][D], mm/ml: [kNW][8] (log2-domain max and
+// running sum).  Called by every thread of the CTA.
+template <int D, typename OutT>
+__device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml, float* wgt,
+                                                float* Ls, float* Ms, int nthreads,
+                                                const DecodeParams& p, int seq, int kvh,
+                                                int part, int n_parts_seq) {
+  const int G = p.group;
+  const int tid = threadIdx.x;
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int w = 0; w < kNW; ++w) M = fmaxf(M, mm[w * 8 + tid]);
+    float L = 0.f;
+    for (int w = 0; w < kNW; ++w) {
+      const float wv = (M == -INFINITY) ? 0.f : exp2f(mm[w * 8 + tid] - M);
+      wgt[w * 8 + tid] = wv;
+      L += wv * ml[w * 8 + tid];
+    }
+    Ls[tid] = L;
+    Ms[tid] = M;
+  }
+  __syncthreads();
+  const size_t head0 = (size_t)seq * p.n_q + (size_t)kvh * G;
+  if (n_parts_seq == 1) {
+    OutT* out = reinterpret_cast<OutT*>(p.out);
+    for (int idx = tid; idx < G * D; idx += nthreads) {
+      const int h = idx / D, dd = idx % D;
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) acc += wgt[w * 8 + h] * mo[(w * 8 + h) * D + dd];
+      const float L = Ls[h];
+      out[(head0 + h) * D + dd] = from_f32<OutT>(L > 0.f ? acc / L * p.out_mul : 0.f);
+    }
+  } else {
+    for (int idx = tid; idx < G * D; idx += nthreads) {
+      const int h = idx / D, dd = idx % D;
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) acc += wgt[w * 8 + h] * mo[(w * 8 + h) * D + dd];
+      p.ws_o[((head0 + h) * p.n_parts_max + part) * D + dd] = acc;
+    }
+    if (tid < G) p.ws_ml[(head0 + tid) * p.n_parts_max + part] = make_float2(Ms[tid], Ls[tid]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core engine: 16-bit caches (MMA in the cache's type) and fp8 caches
+// (MMA in f16); Q_BF16 selects the query / output type.
+// ---------------------------------------------------------------------------
+template <int D, bool FP8, bool Q_BF16>
+__global__ void __launch_bounds__(kThreads) decode_mma_kernel(
+    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+    const DecodeParams p) {
+  using L = MmaLayout<D, FP8>;
+  using QT = typename std::conditional<Q_BF16, __nv_bfloat16, __half>::type;
+  constexpr bool kMmaBf16 = Q_BF16 && !FP8;
+  constexpr int KS = D / 16;  // 16-wide k steps over the head dim / m tiles of O^T
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  const int part = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int G = p.group;
+  const int ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
+                            threadIdx.x == 0 && part == 0 && kvh == 0);
+  const int tok0 = part * kPart;
+  if (tok0 >= ctx) {
+    if (part == 0) {  // empty context: an all-zero output row
+      QT* out = reinterpret_cast<QT*>(p.out);
+      const size_t head0 = (size_t)seq * p.n_q + (size_t)kvh * G;
+      for (int idx = threadIdx.x; idx < G * D; idx += kThreads)
+        out[head0 * D + idx] = from_f32<QT>(0.f);
+    }
+    return;
+  }
+  const int ntok = min(kPart, ctx - tok0);
+  const int nblk = (ntok + 15) >> 4;
+  const int n_parts_seq = (ctx + kPart - 1) / kPart;
+
+  int32_t* ids = reinterpret_cast<int32_t*>(smem + L::kIdsOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + kStages;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x < nblk) {
+    int id = p.block_tables[(size_t)seq * p.max_blocks + (tok0 >> 4) + threadIdx.x];
+    if (id < 0 || id >= p.num_blocks) {
+      flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+      id = -1;
+    }
+    ids[threadIdx.x] = id;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[KS][4];
+#pragma unroll
+  for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  const int g = lane >> 2, t = lane & 3;
+
+  if (warp == kNW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+      const uint64_t pol = l2_policy_evict_first();
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages && !mbar_wait(&empty[s], ((j / kStages) - 1) & 1)) {
+          flag_error(p.dev_err, PA_DEVERR_TIMEOUT);
+          break;
+        }
+        const int id = ids[j];
+        uint8_t* kt = smem + s * L::kStageBytes;
+        uint8_t* vt = kt + L::kTileBytes;
+        if (id >= 0) {
+          mbar_arrive_expect_tx(&full[s], 2 * L::kTileBytes);
+          const int row = (id * p.n_kv + kvh) * 16;
+          if (FP8 || D == 64) {
+            tma_load_2d_hint(kt, &tmk, &full[s], 0, row, pol);
+            tma_load_2d_hint(vt, &tmv, &full[s], 0, row, pol);
+          } else {
+            tma_load_2d_hint(kt, &tmk, &full[s], 0, row, pol);
+            tma_load_2d_hint(kt + 2048, &tmk, &full[s], 64, row, pol);
+            tma_load_2d_hint(vt, &tmv, &full[s], 0, row, pol);
+            tma_load_2d_hint(vt + 2048, &tmv, &full[s], 64, row, pol);
+          }
+        } else {
+          mbar_arrive(&full[s]);
+        }
+        issued = j + 1;
+      }
+      // Before the ring is reused as merge scratch, make sure no load issued
+      // here is still landing (only matters if a consumer gave up early).
+      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        mbar_wait(&full[j % kStages], (j / kStages) & 1);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    // Q as the B operand (k = head dim, n = query head of the group); heads
+    // beyond the group size are zero.  The fp8 path pairs MMA k-index
+    // (2t, 2t+1 | 2t+8, 2t+9) with dims (4t, 4t+1 | 4t+2, 4t+3) of each
+    // 16-dim step so that K can be read as whole 32-bit words; Q uses the
+    // same pairing, which leaves the dot products unchanged.
+    uint32_t qb[KS][2];
+    {
+      const bool hv = g < G;
+      const QT* qrow = reinterpret_cast<const QT*>(p.q) +
+                       ((size_t)seq * p.n_q + (size_t)kvh * G + (hv ? g : 0)) * D;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        if constexpr (FP8) {
+          const int d0 = 16 * kk + 4 * t;
+          qb[kk][0] = pack2<false>(to_f32(qrow[d0]), to_f32(qrow[d0 + 1]));
+          qb[kk][1] = pack2<false>(to_f32(qrow[d0 + 2]), to_f32(qrow[d0 + 3]));
+        } else {
+          qb[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t);
+          qb[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * t);
+        }
+        if (!hv) qb[kk][0] = qb[kk][1] = 0u;
+      }
+    }
+    const float sl = p.scale_log2;
+    const uint32_t sbase = smem_u32(smem);
+    uint8_t* conv = smem + L::kConvOff + warp * L::kConvBytes;
+    const int q4 = lane >> 3;
+
+    for (int j = warp; j < nblk; j += kNW) {
+      const int s = j % kStages;
+      if (!mbar_wait(&full[s], (j / kStages) & 1)) {
+        flag_error(p.dev_err, PA_DEVERR_TIMEOUT);
+        break;
+      }
+      if (ids[j] >= 0) {
+        const int valid = min(16, ntok - 16 * j);
+        const uint32_t kt = sbase + s * L::kStageBytes;
+        // ---- scores S^T = K . Q^T  (16 tokens x 8 heads)
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (!FP8) {
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            const int row = (lane & 7) + ((q4 & 1) << 3);
+            const int C = 2 * kk + (q4 >> 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kt + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2, a3);
+            mma_16816<kMmaBf16>(sc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+          }
+        } else {
+          const uint8_t* ktp = smem + s * L::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < KS; ++kk) {
+            const uint32_t o0 = g * D + 16 * kk + 4 * t, o1 = (g + 8) * D + 16 * kk + 4 * t;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(
+                ktp + (D == 128 ? swz128(o0) : swz64(o0)));
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(
+                ktp + (D == 128 ? swz128(o1) : swz64(o1)));
+            mma_16816<false>(sc, e4m3x2_to_f16x2(w0 & 0xffffu), e4m3x2_to_f16x2(w1 & 0xffffu),
+                             e4m3x2_to_f16x2(w0 >> 16), e4m3x2_to_f16x2(w1 >> 16), qb[kk][0],
+                             qb[kk][1]);
+          }
+        }
+        // ---- online softmax (log2 domain); lane holds tokens g, g+8 of heads 2t, 2t+1
+        float x0 = sc[0] * sl, x1 = sc[1] * sl, x2 = sc[2] * sl, x3 = sc[3] * sl;
+        if (valid < 16) {
+          if (g >= valid) x0 = x1 = -INFINITY;
+          if (g + 8 >= valid) x2 = x3 = -INFINITY;
+        }
+        float b0m = fmaxf(x0, x2), b1m = fmaxf(x1, x3);
+        b0m = warp_max_xor(b0m, 4);
+        b1m = warp_max_xor(b1m, 4);
+        const float n0 = fmaxf(m0, b0m), n1 = fmaxf(m1, b1m);
+        const float c0 = exp2f(m0 - n0), c1 = exp2f(m1 - n1);
+        const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1);
+        const float p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
+        l0 = l0 * c0 + (p0 + p2);
+        l1 = l1 * c1 + (p1 + p3);
+        m0 = n0;
+        m1 = n1;
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+          o[i][0] *= c0;
+          o[i][1] *= c1;
+          o[i][2] *= c0;
+          o[i][3] *= c1;
+        }
+        // P^T as the B operand: transpose the two 8x8 (token x head) halves
+        const uint32_t pb0 = movmatrix_t(pack2<kMmaBf16>(p0, p1));
+        const uint32_t pb1 = movmatrix_t(pack2<kMmaBf16>(p2, p3));
+        // ---- V^T tiles (A operand), O^T += V^T . P^T
+        uint32_t vbase;
+        uint32_t mk01 = 0xffffffffu, mk23 = 0xffffffffu;
+        if constexpr (FP8) {
+          // widen the fp8 V tile to f16 in this warp's tile, zeroing rows
+          // past the context (their bytes are not part of the sequence)
+          const uint8_t* vsrc = smem + s * L::kStageBytes + L::kTileBytes;
+          constexpr int CH = D / 16;
+          __syncwarp();
+#pragma unroll
+          for (int ci = lane; ci < 16 * CH; ci += 32) {
+            const int r = ci / CH, pc = ci % CH;
+            const int lc = (D == 128) ? (pc ^ (r & 7)) : (pc ^ ((r >> 1) & 3));
+            uint4 raw = *reinterpret_cast<const uint4*>(vsrc + r * D + pc * 16);
+            uint32_t h[8];
+            if (r < valid) {
+              h[0] = e4m3x2_to_f16x2(raw.x & 0xffffu);
+              h[1] = e4m3x2_to_f16x2(raw.x >> 16);
+              h[2] = e4m3x2_to_f16x2(raw.y & 0xffffu);
+              h[3] = e4m3x2_to_f16x2(raw.y >> 16);
+              h[4] = e4m3x2_to_f16x2(raw.z & 0xffffu);
+              h[5] = e4m3x2_to_f16x2(raw.z >> 16);
+              h[6] = e4m3x2_to_f16x2(raw.w & 0xffffu);
+              h[7] = e4m3x2_to_f16x2(raw.w >> 16);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) h[e] = 0u;
+            }
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+              const int C = 2 * lc + c2;
+              *reinterpret_cast<uint4*>(conv + swz128((C >> 3) * 2048 + r * 128 + (C & 7) * 16)) =
+                  make_uint4(h[4 * c2], h[4 * c2 + 1], h[4 * c2 + 2], h[4 * c2 + 3]);
+            }
+          }
+          __syncwarp();
+          vbase = smem_u32(conv);
+        } else {
+          vbase = kt + L::kTileBytes;
+          if (valid < 16) {
+            mk01 = ((2 * t < valid) ? 0x0000ffffu : 0u) | ((2 * t + 1 < valid) ? 0xffff0000u : 0u);
+            mk23 = ((2 * t + 8 < valid) ? 0x0000ffffu : 0u) |
+                   ((2 * t + 9 < valid) ? 0xffff0000u : 0u);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+          const int row = (lane & 7) + ((q4 >> 1) << 3);
+          const int C = 2 * i + (q4 & 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vbase + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2, a3);
+          mma_16816<kMmaBf16>(o[i], a0 & mk01, a1 & mk01, a2 & mk23, a3 & mk23, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 4);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 8);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 16);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 4);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 8);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 16);
+  }
+  __syncthreads();  // ring free: reuse it as merge scratch
+
+  float* mo = reinterpret_cast<float*>(smem);
+  float* mm = mo + kNW * 8 * D;
+  float* ml = mm + kNW * 8;
+  float* wgt = ml + kNW * 8;
+  float* Ls = wgt + kNW * 8;
+  float* Ms = Ls + 8;
+  if (warp < kNW) {
+    float* mw = mo + warp * 8 * D;
+#pragma unroll
+    for (int i = 0; i < KS; ++i) {
+      mw[(2 * t) * D + 16 * i + g] = o[i][0];
+      mw[(2 * t + 1) * D + 16 * i + g] = o[i][1];
+      mw[(2 * t) * D + 16 * i + g + 8] = o[i][2];
+      mw[(2 * t + 1) * D + 16 * i + g + 8] = o[i][3];
+    }
+    if (g == 0) {
+      mm[warp * 8 + 2 * t] = m0;
+      mm[warp * 8 + 2 * t + 1] = m1;
+      ml[warp * 8 + 2 * t] = l0;
+      ml[warp * 8 + 2 * t + 1] = l1;
+    }
+  }
+  __syncthreads();
+  merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, part, n_parts_seq);
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core engine for fp32 inputs (exact fp32 arithmetic; small workloads).
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeParams p) {
+  constexpr int VPL = D / 32;  // dims per lane
+  __shared__ int32_t ids[kPartBlocks];
+  __shared__ float mo[kNW * 8 * D];
+  __shared__ float mm[kNW * 8], ml[kNW * 8], wgt[kNW * 8], Ls[8], Ms[8];
+
+  const int part = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int G = p.group;
+  const int ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
+                            threadIdx.x == 0 && part == 0 && kvh == 0);
+  const int tok0 = part * kPart;
+  if (tok0 >= ctx) {
+    if (part == 0) {
+      float* out = reinterpret_cast<float*>(p.out);
+      const size_t head0 = (size_t)seq * p.n_q + (size_t)kvh * G;
+      for (int idx = threadIdx.x; idx < G * D; idx += kNW * 32) out[head0 * D + idx] = 0.f;
+    }
+    return;
+  }
+  const int ntok = min(kPart, ctx - tok0);
+  const int nblk = (ntok + 15) >> 4;
+  const int n_parts_seq = (ctx + kPart - 1) / kPart;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < nblk) {
+    int id = p.block_tables[(size_t)seq * p.max_blocks + (tok0 >> 4) + threadIdx.x];
+    if (id < 0 || id >= p.num_blocks) {
+      flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+      id = -1;
+    }
+    ids[threadIdx.x] = id;
+  }
+  __syncthreads();
+
+  const float* qp = reinterpret_cast<const float*>(p.q) + ((size_t)seq * p.n_q + (size_t)kvh * G) * D;
+  float qv[kMaxGroup][VPL], o[kMaxGroup][VPL], m[kMaxGroup], l[kMaxGroup];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      qv[h][i] = h < G ? qp[h * D + lane * VPL + i] : 0.f;
+      o[h][i] = 0.f;
+    }
+  }
+  const float* kpool = reinterpret_cast<const float*>(p.k_pool);
+  const float* vpool = reinterpret_cast<const float*>(p.v_pool);
+  for (int j = warp; j < nblk; j += kNW) {
+    const int id = ids[j];
+    if (id < 0) continue;
+    const int valid = min(16, ntok - 16 * j);
+    const size_t base = ((size_t)id * p.n_kv + kvh) * 16 * D;
+    for (int tt = 0; tt < valid; ++tt) {
+      float kr[VPL], vr[VPL];
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        kr[i] = kpool[base + tt * D + lane * VPL + i];
+        vr[i] = vpool[base + tt * D + lane * VPL + i];
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) {
+        if (h >= G) break;
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) s = fmaf(qv[h][i], kr[i], s);
+#pragma unroll
+        for (int msk = 16; msk >= 1; msk >>= 1) s += __shfl_xor_sync(0xffffffffu, s, msk);
+        s *= p.scale_log2;
+        const float mn = fmaxf(m[h], s);
+        const float c = exp2f(m[h] - mn), pr = exp2f(s - mn);
+        l[h] = l[h] * c + pr;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) o[h][i] = fmaf(pr, vr[i], o[h][i] * c);
+        m[h] = mn;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) mo[(warp * 8 + h) * D + lane * VPL + i] = o[h][i];
+    if (lane == 0) {
+      mm[warp * 8 + h] = m[h];
+      ml[warp * 8 + h] = l[h];
+    }
+  }
+  __syncthreads();
+  merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, part, n_parts_seq);
+}
+
+// ---------------------------------------------------------------------------
+// partition merge: one warp per (sequence, q head) with more than one
+// partition; partitions combined in increasing order.
+// ---------------------------------------------------------------------------
+template <int D, typename OutT>
+__global__ void __launch_bounds__(256) decode_reduce_kernel(const ReduceParams r) {
+  constexpr int VPL = D / 32;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= r.num_seqs * r.n_q) return;
+  const int seq = gw / r.n_q;
+  int ctx = r.context_lens[seq];
+  ctx = ctx < 0 ? 0 : min(ctx, r.max_blocks * 16);
+  const int np = (ctx + kPart - 1) / kPart;
+  if (np <= 1) return;
+  const float2* ml = r.ws_ml + (size_t)gw * r.n_parts_max;
+  float M = -INFINITY;
+  for (int pp = lane; pp < np; pp += 32) M = fmaxf(M, ml[pp].x);
+  M = warp_max_xor(M, 1);
+  float L = 0.f, acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  const float* wo = r.ws_o + (size_t)gw * r.n_parts_max * D + lane * VPL;
+  for (int pp = 0; pp < np; ++pp) {
+    const float2 v = ml[pp];
+    const float w = (v.x == -INFINITY) ? 0.f : exp2f(v.x - M);
+    L += w * v.y;
+    if constexpr (VPL == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(wo + (size_t)pp * D);
+      acc[0] += w * x.x;
+      acc[1] += w * x.y;
+      acc[2] += w * x.z;
+      acc[3] += w * x.w;
+    } else {
+      const float2 x = *reinterpret_cast<const float2*>(wo + (size_t)pp * D);
+      acc[0] += w * x.x;
+      acc[1] += w * x.y;
+    }
+  }
+  OutT* out = reinterpret_cast<OutT*>(r.out) + (size_t)gw * D + lane * VPL;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) out[i] = from_f32<OutT>(L > 0.f ? acc[i] / L * r.out_mul : 0.f);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D, bool FP8, bool Q_BF16>
+cudaError_t launch_mma(const DecodeParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                       cudaStream_t st) {
+  using L = MmaLayout<D, FP8>;
+  static cudaError_t attr = set_smem(decode_mma_kernel<D, FP8, Q_BF16>, L::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  dim3 grid(p.n_parts_max, p.n_kv, p.num_seqs);
+  decode_mma_kernel<D, FP8, Q_BF16><<<grid, kThreads, L::kSmemBytes, st>>>(*tmk, *tmv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_simt(const DecodeParams& p, cudaStream_t st) {
+  dim3 grid(p.n_parts_max, p.n_kv, p.num_seqs);
+  decode_simt_f32_kernel<D><<<grid, kNW * 32, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_num_parts(int max_blocks_per_seq) {
+  return (max_blocks_per_seq * 16 + kPart - 1) / kPart;
+}
+
+bool decode_uses_tma(pa_dtype q_dt, pa_dtype kv_dt) { return q_dt != PA_F32; }
+
+cudaError_t launch_decode_partitions(const DecodeParams& p, int D, pa_dtype q_dt,
+                                     pa_dtype kv_dt, const CUtensorMap* tmk,
+                                     const CUtensorMap* tmv, cudaStream_t st) {
+  const bool fp8 = kv_dt == PA_FP8_E4M3;
+  if (q_dt == PA_F32) return D == 64 ? launch_simt<64>(p, st) : launch_simt<128>(p, st);
+  if (q_dt == PA_BF16) {
+    if (fp8) return D == 64 ? launch_mma<64, true, true>(p, tmk, tmv, st)
+                            : launch_mma<128, true, true>(p, tmk, tmv, st);
+    return D == 64 ? launch_mma<64, false, true>(p, tmk, tmv, st)
+                   : launch_mma<128, false, true>(p, tmk, tmv, st);
+  }
+  if (fp8) return D == 64 ? launch_mma<64, true, false>(p, tmk, tmv, st)
+                          : launch_mma<128, true, false>(p, tmk, tmv, st);
+  return D == 64 ? launch_mma<64, false, false>(p, tmk, tmv, st)
+                 : launch_mma<128, false, false>(p, tmk, tmv, st);
+}
+
+cudaError_t launch_decode_reduce(const ReduceParams& r, int D, pa_dtype out_dt,
+                                 cudaStream_t st) {
+  const int blocks = (r.num_seqs * r.n_q + 7) / 8;
+  if (blocks == 0) return cudaSuccess;
+#define PA_RED(DD, T) decode_reduce_kernel<DD, T><<<blocks, 256, 0, st>>>(r)
+  if (out_dt == PA_F32) {
+    if (D == 64) PA_RED(64, float); else PA_RED(128, float);
+  } else if (out_dt == PA_BF16) {
+    if (D == 64) PA_RED(64, __nv_bfloat16); else PA_RED(128, __nv_bfloat16);
+  } else {
+    if (D == 64) PA_RED(64, __half); else PA_RED(128, __half);
+  }
+#undef PA_RED
+  return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,103 @@
+"""The C ABI library loads without a GPU, exports every symbol include/pa.h
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    from pagedattention_paged_kv_pa_b200 import build
+    build.build()
+    from pagedattention_paged_kv_pa_b200 import binding
+    return binding
+
+
+def test_header_declares_the_hot_path_calls():
+    names = _declared()
+    for n in ("pa_decode", "pa_reshape_and_cache", "pa_copy_blocks", "pa_prefill_paged",
+              "pa_alloc_create", "pa_alloc_prepare_write"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(B):
+    names = _declared()
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(l.split()[-1] for l in out.splitlines() if " T " in l)
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert set(B.EXPORTS) == set(names)
+
+
+def test_library_needs_no_cuda_driver_to_load(B):
+    out = subprocess.run(["ldd", B.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out  # driver entry points are fetched at run time
+    assert B.lib.pa_abi_version() == 1
+
+
+def test_status_strings(B):
+    assert B.status_string(0) == "ok"
+    assert "unsupported" in B.status_string(2)
+
+
+def _dec(B, **kw):
+    a = dict(out=16, q=16, k=16, v=16, bt=16, cl=16, scale=0.1, bs=16, nq=8, nkv=2, d=128,
+             ns=4, mb=4, nb=10, qdt=B.PA_BF16, kvdt=B.PA_BF16, ks=1.0, vs=1.0, ws=None,
+             wsb=0, err=None, st=None)
+    a.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return B.lib.pa_decode(v(a["out"]), v(a["q"]), v(a["k"]), v(a["v"]), v(a["bt"]), v(a["cl"]),
+                           a["scale"], a["bs"], a["nq"], a["nkv"], a["d"], a["ns"], a["mb"],
+                           a["nb"], a["qdt"], a["kvdt"], a["ks"], a["vs"], v(a["ws"]), a["wsb"],
+                           v(a["err"]), v(a["st"]))
+
+
+def test_decode_argument_errors_are_synchronous(B):
+    # none of these reach a launch, so they are safe without a GPU
+    assert _dec(B, bs=32) == B.PA_ERR_UNSUPPORTED
+    assert _dec(B, d=96) == B.PA_ERR_UNSUPPORTED
+    assert _dec(B, nq=6, nkv=4) == B.PA_ERR_INVALID_ARG
+    assert _dec(B, nq=32, nkv=2) == B.PA_ERR_UNSUPPORTED          # group 16 > 8
+    assert _dec(B, qdt=B.PA_F32, kvdt=B.PA_BF16) == B.PA_ERR_UNSUPPORTED
+    assert _dec(B, qdt=B.PA_FP8_E4M3, kvdt=B.PA_FP8_E4M3) == B.PA_ERR_UNSUPPORTED
+    assert _dec(B, q=None) == B.PA_ERR_INVALID_ARG
+    assert _dec(B, q=24) == B.PA_ERR_INVALID_ARG                  # misaligned pointer
+    assert _dec(B, mb=0) == B.PA_ERR_INVALID_ARG
+    assert _dec(B, ns=0) == B.PA_OK                               # nothing to do
+    # more than one partition needs a workspace of the advertised size
+    ws = B.pa_decode_workspace_size(4, 8, 128, 512)
+    assert ws > 0
+    assert _dec(B, mb=512) == B.PA_ERR_INVALID_ARG
+    assert _dec(B, mb=512, ws=16, wsb=ws - 1) == B.PA_ERR_INVALID_ARG
+    assert _dec(B, kvdt=B.PA_FP8_E4M3, ks=0.0) == B.PA_ERR_INVALID_ARG
+    assert B.pa_decode_workspace_size(4, 8, 128, 32) == 0          # a single partition
+
+
+def test_cache_op_argument_errors_are_synchronous(B):
+    v = ctypes.c_void_p
+    L = B.lib
+    assert L.pa_reshape_and_cache(v(16), v(16), v(16), v(16), v(16), 4, 2, 128, 8, 10,
+                                  B.PA_BF16, B.PA_BF16, 1.0, 1.0, None, None) == B.PA_ERR_UNSUPPORTED
+    assert L.pa_reshape_and_cache(v(16), v(16), v(16), v(16), v(16), 4, 2, 128, 16, 10,
+                                  B.PA_BF16, B.PA_F16, 1.0, 1.0, None, None) == B.PA_ERR_UNSUPPORTED
+    assert L.pa_reshape_and_cache(v(16), v(16), v(16), v(16), v(16), 4, 2, 128, 16, 10,
+                                  B.PA_BF16, B.PA_FP8_E4M3, 0.0, 1.0, None, None) == B.PA_ERR_INVALID_ARG
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 2, 128, 16, 10,
+                                  B.PA_BF16, B.PA_BF16, 1.0, 1.0, None, None) == B.PA_OK
+    assert L.pa_copy_blocks(v(16), v(16), None, 3, 8, 128, 16, 10, B.PA_BF16, None,
+                            None) == B.PA_ERR_INVALID_ARG
+    assert L.pa_copy_blocks(None, None, None, 0, 8, 128, 16, 10, B.PA_BF16, None,
+                            None) == B.PA_OK
