@@ -139,6 +139,39 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
                            pa_dtype q_dtype, pa_dtype kv_dtype, float v_scale,
                            const void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory and therefore have no workspace to pass: for example a plugin inside
+ * a host program that owns all device memory and forbids cudaMalloc after
+ * start-up, or a loop that cannot afford cudaMalloc's implicit device
+ * synchronisation.  The pages have no counterpart to this: it is a packaging
+ * of pa_decode, not part of the method.
+ *
+ * Same arguments and results as pa_decode without the workspace.  The
+ * per-partition results go to a scratch array built into the library (a
+ * file-scope __device__ array of pa_decode_noalloc_scratch_bytes() = 16 MiB;
+ * every GPU that loads the library holds it until the process exits).  The
+ * call makes no cudaMalloc, cudaFree or other allocating call.
+ *  - Returns PA_ERR_UNSUPPORTED before any launch when the call would need more
+ *    scratch than that, i.e. when pa_decode_workspace_size(num_seqs, n_q_heads,
+ *    head_dim, max_blocks_per_seq) > pa_decode_noalloc_scratch_bytes().
+ *  - The first call on a device looks up the array's device address with that
+ *    device current and caches it; make that first call before any stream
+ *    capture.
+ *  - All calls share the one array, which keeps the last call's contents:
+ *    calls whose work overlaps on the GPU (other streams, other host threads)
+ *    race on it and must be ordered by the caller.  Nothing in it needs to
+ *    start at zero.
+ */
+size_t pa_decode_noalloc_scratch_bytes(void);
+
+pa_status pa_decode_noalloc(void* out, const void* q, const void* k_pool, const void* v_pool,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            float scale, int block_size, int n_q_heads, int n_kv_heads,
+                            int head_dim, int num_seqs, int max_blocks_per_seq, int num_blocks,
+                            pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
+                            int32_t* dev_err, void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* Chunked prefill                                                            */
 /* ------------------------------------------------------------------------- */

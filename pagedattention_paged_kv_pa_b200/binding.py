@@ -28,7 +28,7 @@ EXPORTS = (
     "pa_copy_blocks", "pa_alloc_create", "pa_alloc_destroy", "pa_alloc_append",
     "pa_alloc_fork", "pa_alloc_prepare_write", "pa_alloc_free_seq", "pa_alloc_block_table",
     "pa_alloc_free_list", "pa_alloc_num_tokens", "pa_alloc_refcount", "pa_alloc_num_free",
-    "pa_alloc_num_seqs",
+    "pa_alloc_num_seqs", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
 )
 
 
@@ -53,6 +53,9 @@ def _load() -> ctypes.CDLL:
     L.pa_decode.argtypes = dec
     L.pa_decode_partitions.argtypes = dec
     L.pa_decode_reduce.argtypes = [P, P, I, I, I, I, I, I, F, P, Z, P]
+    L.pa_decode_noalloc.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, F, F, P, P]
+    L.pa_decode_noalloc.restype = I
+    L.pa_decode_noalloc_scratch_bytes.restype = Z
     L.pa_prefill_paged.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, F, F,
                                    P, P]
     L.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, F, P, P]
@@ -158,6 +161,25 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale
     _check(lib.pa_decode(*_decode_args(out, q, k_pool, v_pool, block_tables, context_lens,
                                        scale, k_scale, v_scale, workspace, dev_err, stream)),
            "pa_decode")
+    return out
+
+
+def pa_decode_noalloc(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale=1.0,
+                      v_scale=1.0, dev_err=None, stream=None):
+    """pa_decode without a caller workspace: the library's own static device
+    scratch holds the partition results (see include/pa.h for its limit and
+    the ordering rule between calls)."""
+    a = _decode_args(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale,
+                     v_scale, None, dev_err, stream)
+    st = lib.pa_decode_noalloc(*a[:18], a[20], a[21])
+    if st == PA_ERR_UNSUPPORTED:
+        need = pa_decode_workspace_size(q.shape[0], q.shape[1], q.shape[2],
+                                        block_tables.shape[1])
+        cap = lib.pa_decode_noalloc_scratch_bytes()
+        if need > cap:
+            raise PAError(st, f"pa_decode_noalloc needs {need} bytes of scratch; the library's "
+                              f"static scratch holds {cap}")
+    _check(st, "pa_decode_noalloc")
     return out
 
 
