@@ -357,17 +357,20 @@ def run_ours(args, rank, world, local):
 
 def traffic_from_profile(workload):
     """DRAM bytes per launch of the partition kernel from the committed ncu
-    summary, if that summary matches the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    summary (profiles/decode_traffic.txt), if that summary was taken on the
+    current kernel source; None otherwise."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+    src = os.path.join(ROOT, "pagedattention_paged_kv_pa_b200", "csrc", "decode.cu")
     try:
-        with open(path) as f:
-            rec = json.load(f)
-        src = os.path.join(ROOT, "pagedattention_paged_kv_pa_b200", "csrc", "decode.cu")
-        import hashlib
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if rec.get("decode_cu_sha256_16") != h:
+        rec = {}
+        for line in open(path):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                rec[k.strip()] = v.strip()
+        if rec.get("decode_cu_sha256_16") != hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]:
             return None
-        return rec.get("traffic_bytes_per_launch", {}).get(workload)
+        return int(rec[workload]) if workload in rec else None
     except Exception:
         return None
 
