@@ -355,6 +355,169 @@ def run_ours(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def prefill_causal_flops(inp) -> int:
+    """Algorithmic flops of causal chunked prefill: 2 products x 2 flop x d per
+    (query row, q head, visible key)."""
+    qsl = inp.query_start_loc.cpu().numpy()
+    cl = inp.context_lens.cpu().numpy()
+    keys = 0
+    for c in range(len(cl)):
+        L = int(qsl[c + 1] - qsl[c])
+        H = int(cl[c]) - L
+        keys += L * H + L * (L + 1) // 2
+    s = inp.spec
+    return 4 * s.head_dim * s.n_q_heads * keys
+
+
+def run_mixed(args, rank, world, local):
+    """Mixed continuous-batching step: slot writes of all new tokens, then the
+    decode (256 sequences) on one stream and the chunked prefill (2 chunks of
+    512 queries over 4096 tokens of history) on another, fp8 KV cache."""
+    import torch
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_init(world, "nccl")
+    dspec, pspec = W.MIXED_DECODE_FP8, W.MIXED_PREFILL_FP8
+    dinp = W.make_decode_inputs(dspec, device=dev)
+    pinp = W.make_prefill_inputs(pspec, device=dev)
+    ctx = dinp.context_lens.cpu().numpy()
+    n = dspec.num_seqs
+    # new tokens: one per decode sequence, the whole chunk for each prefill
+    dkey, dval = W.make_new_kv(n, dspec.n_kv_heads, dspec.head_dim, W.BF16, dev, seed=3005)
+    dslots = torch.from_numpy(W.slots_from_positions(
+        dinp.block_tables.cpu().numpy(), np.arange(n), ctx - 1)).to(dev)
+    qsl = pinp.query_start_loc.cpu().numpy()
+    pcl = pinp.context_lens.cpu().numpy()
+    seq_ids = np.concatenate([np.full(int(qsl[c + 1] - qsl[c]), c) for c in range(len(pcl))])
+    pos = np.concatenate([np.arange(int(pcl[c]) - int(qsl[c + 1] - qsl[c]), int(pcl[c]))
+                          for c in range(len(pcl))])
+    pslots = torch.from_numpy(W.slots_from_positions(pinp.block_tables.cpu().numpy(), seq_ids,
+                                                     pos)).to(dev)
+    pkey, pval = W.make_new_kv(len(pos), pspec.n_kv_heads, pspec.head_dim, W.BF16, dev,
+                               seed=3006)
+    dout = torch.empty_like(dinp.q)
+    pout = torch.empty_like(pinp.q)
+    mb = dinp.block_tables.shape[1]
+    ws = B.alloc_decode_workspace(dinp.q, mb)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    s_dec = torch.cuda.current_stream(dev)
+    s_pre = torch.cuda.Stream(dev)
+    dec_bytes = W.decode_algorithmic_bytes(ctx, dspec.n_q_heads, dspec.n_kv_heads,
+                                           dspec.head_dim, 2, 1)
+    flops = prefill_causal_flops(pinp)
+
+    def decode_part(ev=None):
+        B.pa_reshape_and_cache(dinp.k_pool, dinp.v_pool, dkey, dval, dslots, dinp.k_scale,
+                               dinp.v_scale, dev_err=err, stream=s_dec)
+        if ev is not None:
+            ev[0].record(s_dec)
+        B.pa_decode_partitions(dout, dinp.q, dinp.k_pool, dinp.v_pool, dinp.block_tables,
+                               dinp.context_lens, dinp.scale, dinp.k_scale, dinp.v_scale,
+                               workspace=ws, dev_err=err, stream=s_dec)
+        if ev is not None:
+            ev[1].record(s_dec)
+        B.pa_decode_reduce(dout, dinp.context_lens, mb, B.PA_FP8_E4M3, dinp.v_scale,
+                           workspace=ws, stream=s_dec)
+
+    def prefill_part(ev=None):
+        B.pa_reshape_and_cache(pinp.k_pool, pinp.v_pool, pkey, pval, pslots, pinp.k_scale,
+                               pinp.v_scale, dev_err=err, stream=s_pre)
+        if ev is not None:
+            ev[0].record(s_pre)
+        B.pa_prefill_paged(pout, pinp.q, pinp.k_pool, pinp.v_pool, pinp.block_tables,
+                           pinp.query_start_loc, pinp.context_lens, pinp.scale,
+                           pspec.chunk_len, pinp.k_scale, pinp.v_scale, dev_err=err,
+                           stream=s_pre)
+        if ev is not None:
+            ev[1].record(s_pre)
+
+    def step(dev_ev=None, pre_ev=None):
+        s_pre.wait_stream(s_dec)
+        prefill_part(pre_ev)
+        decode_part(dev_ev)
+        s_dec.wait_stream(s_pre)
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+
+    # each part alone (kernel rooflines), then the concurrent step
+    def time_alone(fn, k):
+        evs = [(mk(), mk()) for _ in range(k)]
+        torch.cuda.synchronize()
+        for i in range(k):
+            fn(evs[i])
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / k
+
+    K = args.steps
+    dec_ms = time_alone(decode_part, min(K, 200))
+    s_pre.wait_stream(s_dec)
+    pre_ms = time_alone(prefill_part, min(K, 200))
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    time.sleep(0.3)
+    t0, t1 = mk(), mk()
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    t0.record(s_dec)
+    for _ in range(K):
+        step()
+    t1.record(s_dec)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clocks = sampler.stop()
+    ms = reduce_over_ranks(t0.elapsed_time(t1), "max", world, dev)
+    value = reduce_over_ranks(dec_bytes * K, "sum", world, dev) / (ms / 1e3) / 1e9
+    peak, _ = hbm_peak()
+    try:
+        tflops_peak = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+        tsrc = "measured bf16_tflops (burst; f16 and bf16 share the nominal 2.25 PF)"
+    except Exception:
+        tflops_peak, tsrc = 1590.0, "fallback 1.59 PF"
+    pre_tflops = flops / (pre_ms / 1e3) / 1e12
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16+fp8kv",
+        "data": "synthetic (seeded N(0,1) values, seeded lengths and block shuffle)",
+        "config": {"workload": "mixed continuous-batching step: " + describe(dspec, ctx, dinp.num_blocks)
+                   + f"; + prefill of 2 chunks x 512 queries over 4096-token paged histories, "
+                     f"32 q / 8 kv heads, fp8 KV; slot writes of all {n + len(pos)} new tokens; "
+                     "decode and prefill on two streams",
+                   "global_batch": n * world, "seq_len": int(ctx.max()),
+                   "l2": "inputs larger than L2 (decode KV 2.2 GB); no flush",
+                   "parallelism": f"replicas x{world}"},
+        "value_counts": "decode algorithmic bytes per concurrent step time",
+        "decode_alone": {"us": round(dec_ms * 1e3, 2), "achieved_gbs": round(dec_gbs, 1),
+                         "frac": round(dec_gbs / peak, 4),
+                         "includes": "slot write + partition kernel"},
+        "prefill_alone": {"us": round(pre_ms * 1e3, 2), "algorithmic_flop": int(flops),
+                          "achieved_tflops": round(pre_tflops, 1),
+                          "peak_tflops": tflops_peak, "frac": round(pre_tflops / tflops_peak, 4),
+                          "peak_source": tsrc, "includes": "slot write + prefill kernel"},
+        "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(dec_gbs / peak, 4), "traffic": None,
+                     "kernel": "decode_mma_kernel (fp8 cache)"},
+        "gpu_launches": 5 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def traffic_from_profile(workload):
     """DRAM bytes per launch of the partition kernel from the committed ncu
     summary (profiles/decode_traffic.txt), if that summary was taken on the
@@ -426,6 +589,8 @@ def main(argv=None):
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world, local)
+    elif args.workload == "mixed_step_fp8":
+        run_mixed(args, rank, world, local)
     else:
         run_ours(args, rank, world, local)
 

@@ -195,9 +195,14 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_pool, const 
  *   context_lens   device int32 [n_chunks], context_lens[c] >= L_c
  *   max_chunk_len  host bound on every L_c (sizes the grid; no device sync)
  *
- * Supported: block_size 16, head_dim 128, group size <= 8, q_dtype BF16 and
- * kv_dtype BF16 or FP8_E4M3 (FP8 K/V are widened to bf16 in shared memory,
- * exactly).  The output is written in q_dtype.
+ * Supported: block_size 16, head_dim 128, group size 1, 2, 4 or 8, q_dtype
+ * BF16 and kv_dtype BF16 or FP8_E4M3.  The products run in f16 with fp32
+ * accumulation: E4M3 values widen to f16 exactly; bf16 q/K/V values are exact
+ * in f16 while |x| <= 65504 (values below 2^-14 keep an absolute precision of
+ * 2^-24; larger magnitudes overflow), a restriction the bf16-cache variant
+ * carries.  A block id outside [0, num_blocks) is flagged with
+ * PA_DEVERR_BLOCK_ID and its keys read as zeros.  The output is written in
+ * q_dtype.
  */
 pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
                            const int32_t* block_tables, const int32_t* query_start_loc,

@@ -267,6 +267,53 @@ pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_
                           q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
 }
 
+pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
+                           const int32_t* block_tables, const int32_t* query_start_loc,
+                           const int32_t* context_lens, float scale, int block_size,
+                           int n_q_heads, int n_kv_heads, int head_dim, int n_chunks,
+                           int max_chunk_len, int max_blocks_per_seq, int num_blocks,
+                           pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
+                           int32_t* dev_err, void* stream) {
+  if (block_size != 16 || head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int G = n_q_heads / n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+  if (n_chunks < 0 || max_chunk_len < 1 || max_blocks_per_seq < 1 || num_blocks < 1)
+    return PA_ERR_INVALID_ARG;
+  if (n_chunks > 65535 || n_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+  if ((int64_t)max_blocks_per_seq * 16 >= (int64_t(1) << 30)) return PA_ERR_UNSUPPORTED;
+  if (q_dtype != PA_BF16 || (kv_dtype != PA_BF16 && kv_dtype != PA_FP8_E4M3))
+    return PA_ERR_UNSUPPORTED;
+  if (!(scale == scale) || (kv_dtype == PA_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)))
+    return PA_ERR_INVALID_ARG;
+  if (n_chunks == 0) return PA_OK;
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !query_start_loc || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
+    return PA_ERR_INVALID_ARG;
+  const int grid_x = (max_chunk_len + (128 / G) - 1) / (128 / G);
+  if (grid_x > 65535 * 32) return PA_ERR_UNSUPPORTED;
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  pa::PrefillParams p;
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.query_start_loc = query_start_loc;
+  p.context_lens = context_lens;
+  p.dev_err = dev_err;
+  p.scale_log2 = scale * kLog2e * (fp8 ? k_scale : 1.f);
+  p.out_mul = fp8 ? v_scale : 1.f;
+  p.n_q = n_q_heads;
+  p.n_kv = n_kv_heads;
+  p.group = G;
+  p.n_chunks = n_chunks;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.max_chunk_len = max_chunk_len;
+  return cuda_status(
+      pa::launch_prefill(p, kv_dtype, k_pool, v_pool, static_cast<cudaStream_t>(stream)));
+}
+
 pa_status pa_reshape_and_cache(void* k_pool, void* v_pool, const void* key, const void* value,
                                const int64_t* slot_mapping, int num_tokens, int n_kv_heads,
                                int head_dim, int block_size, int num_blocks, pa_dtype src_dtype,

@@ -25,7 +25,8 @@
 //
 // Per-block math (16-bit and fp8 caches): S^T[16 tok][8 heads] = K . Q^T and
 // O^T[d][8 heads] += V^T . P^T, each as m16n8k16 warp MMAs with the GQA group
-// as N=8 (fp32 accumulate).  For fp8 caches the E4M3 codes are widened to f16
+// as N=8 (fp32 accumulate; with 16-bit caches P enters as a 16-bit value plus
+// its 16-bit rounding residual).  For fp8 caches the E4M3 codes are widened to f16
 // exactly (K in registers, V through a per-warp shared tile) and the
 // per-tensor scales are applied to the scores and to the final output.  fp32
 // inputs use a CUDA-core path with fp32 arithmetic throughout.
@@ -318,9 +319,19 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
           o[i][2] *= c0;
           o[i][3] *= c1;
         }
-        // P^T as the B operand: transpose the two 8x8 (token x head) halves
-        const uint32_t pb0 = movmatrix_t(pack2<kMmaBf16>(p0, p1));
-        const uint32_t pb1 = movmatrix_t(pack2<kMmaBf16>(p2, p3));
+        // P^T as the B operand: transpose the two 8x8 (token x head) halves.
+        // With 16-bit caches P is split into a rounded part and its rounding
+        // residual (two MMAs), which keeps ~16 significant bits of P: a single
+        // bf16 P would cost up to 2^-9 |v - o| on short contexts.
+        const uint32_t ph01 = pack2<kMmaBf16>(p0, p1), ph23 = pack2<kMmaBf16>(p2, p3);
+        const uint32_t pb0 = movmatrix_t(ph01);
+        const uint32_t pb1 = movmatrix_t(ph23);
+        uint32_t pl0 = 0u, pl1 = 0u;
+        if constexpr (!FP8) {
+          const float2 h01 = unpack2<kMmaBf16>(ph01), h23 = unpack2<kMmaBf16>(ph23);
+          pl0 = movmatrix_t(pack2<kMmaBf16>(p0 - h01.x, p1 - h01.y));
+          pl1 = movmatrix_t(pack2<kMmaBf16>(p2 - h23.x, p3 - h23.y));
+        }
         // ---- V^T tiles (A operand), O^T += V^T . P^T
         uint32_t vbase;
         uint32_t mk01 = 0xffffffffu, mk23 = 0xffffffffu;
@@ -372,7 +383,12 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
           const int C = 2 * i + (q4 & 1);
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(vbase + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2, a3);
-          mma_16816<kMmaBf16>(o[i], a0 & mk01, a1 & mk01, a2 & mk23, a3 & mk23, pb0, pb1);
+          a0 &= mk01;
+          a1 &= mk01;
+          a2 &= mk23;
+          a3 &= mk23;
+          mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pb0, pb1);
+          if constexpr (!FP8) mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pl0, pl1);
         }
       }
       __syncwarp();

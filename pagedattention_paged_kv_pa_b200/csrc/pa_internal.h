@@ -80,7 +80,7 @@ struct PrefillParams {
   float out_mul;
   int n_q, n_kv, group, n_chunks, max_blocks, num_blocks, max_chunk_len;
 };
-cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const CUtensorMap* tmq,
-                           const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st);
+cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k_pool,
+                           const void* v_pool, cudaStream_t st);
 
 }  // namespace pa

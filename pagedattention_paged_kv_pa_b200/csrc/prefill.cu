@@ -1,9 +1,497 @@
-// Chunked prefill over the paged cache (tcgen05).  Entry point only for now.
+// Chunked prefill over the paged cache on tcgen05 tensor cores (sm_100a).
+//
+// A long prompt is cut into chunks that run next to decodes ("LLM inference
+// optimization: KV cache & PagedAttention", §六.2; "vLLM explained",
+// "附錄與延伸").  Chunk c holds L queries at absolute positions H..H+L-1 over
+// a paged history of H tokens; query i attends causally to keys 0..H+i.  With
+// many queries per chunk the two products are real dense contractions, so
+// they run on the 5th-generation tensor cores with accumulators in TMEM.
+//
+// CTA tile: M = 128 rows = (128 / G) consecutive queries x the G query heads
+// of one kv head (GQA packing: each K/V tile is widened once for the whole
+// group).  Keys are processed in tiles of 128 (8 blocks of 16 from the block
+// table).  Warp roles (288 threads):
+//   warps 0-3  softmax: thread r owns row r = TMEM lane r; reads S from TMEM,
+//              masks, keeps an online max/sum, writes P (16-bit) to shared
+//              memory, rescales the TMEM output when its max grew by more
+//              than 2^8, and writes the normalised output at the end;
+//   warps 4-7  K/V converters: load a tile's K and V rows through the block
+//              table with coalesced 16-byte loads, widen fp8 codes exactly to
+//              f16 (bf16 values are converted to f16), write K in the K-major
+//              128-byte-swizzled layout the MMA reads and V transposed (V^T,
+//              also K-major);
+//   warp 8     TMEM owner and MMA issuer (one elected lane): S = Q K^T into a
+//              double-buffered TMEM score tile, O += P V into TMEM.
+// Both MMAs run in f16 with fp32 accumulation: every E4M3 value is exact in
+// f16, bf16 inputs are exact while inside f16's range (|x| <= 65504; below
+// 2^-14 they keep an absolute precision of 2^-24), and P gets 11 significant
+// bits instead of bf16's 8.
+// S(j+1) is issued before O += P(j) V(j), so the next tile's QK^T overlaps
+// this tile's softmax; K/V operands are double buffered.  All waits are
+// bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA drains its
+// tensor-core work and frees its TMEM before returning.
+#include "pa_device.cuh"
 #include "pa_internal.h"
 
-extern "C" pa_status pa_prefill_paged(void*, const void*, const void*, const void*,
-                                      const int32_t*, const int32_t*, const int32_t*, float,
-                                      int, int, int, int, int, int, int, int, pa_dtype,
-                                      pa_dtype, float, float, int32_t*, void*) {
-  return PA_ERR_UNSUPPORTED;
+namespace pa {
+
+namespace {
+
+constexpr int D = 128;       // head dim
+constexpr int BM = 128;      // rows per CTA tile
+constexpr int BN = 128;      // keys per tile
+constexpr int kThreads = 288;
+constexpr int kSoftmaxWarps = 4, kMmaWarp = 8;  // warps 4-7 convert K/V
+constexpr uint32_t kTmemCols = 512;  // S[2] x 128 + O 128 -> 384, rounded to 2^k
+constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
+
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr int kOpBytes = BM * D * 2;  // one 128x128 16-bit operand = 32 KiB
+constexpr int kQOff = 0;
+constexpr int kKOff = kQOff + kOpBytes;       // 2 stages
+constexpr int kVOff = kKOff + 2 * kOpBytes;   // 2 stages (V^T)
+constexpr int kPOff = kVOff + 2 * kOpBytes;
+constexpr int kStgOff = kPOff + kOpBytes;     // widened V, [key][d], 256-B rows
+constexpr int kBarOff = kStgOff + kOpBytes;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;
+
+// K-major operand with 128-byte swizzle: rows of 64 16-bit elements (128 B)
+// in two 16 KiB halves along K; chunk = 8 elements along K (0..15).
+__device__ __forceinline__ uint32_t op_off(int row, int chunk) {
+  return (chunk >> 3) * 16384 + row * 128 + ((((chunk & 7) ^ (row & 7))) << 4);
 }
+// staging [key][d] with the 32-byte granule XOR-ed by (key & 7)
+__device__ __forceinline__ uint32_t stg_off(int key, int d) {
+  return key * 256 + ((((d >> 4) ^ (key & 7))) << 5) + ((d & 15) << 1);
+}
+
+// ------------------------------------------------------------- tcgen05 ops
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void conv_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// barrier over the 128 converter threads that also ORs a flag across them
+__device__ __forceinline__ bool conv_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+struct Bars {
+  uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, pv_done, done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// bounded wait that also honours the CTA-wide abort flag
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Bars* B,
+                                              int32_t* dev_err) {
+  if (mbar_wait(bar, parity)) return true;
+  flag_error(dev_err, PA_DEVERR_TIMEOUT);
+  *reinterpret_cast<volatile int*>(&B->abort_flag) = 1;
+  return false;
+}
+__device__ __forceinline__ bool aborted(Bars* B) {
+  return *reinterpret_cast<volatile int*>(&B->abort_flag) != 0;
+}
+
+// bf16x2 -> f16x2 (exact for values inside f16's normal range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  return pack2<false>(f.x, f.y);
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const PrefillParams p, const void* __restrict__ k_pool,
+                      const void* __restrict__ v_pool) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  Bars* B = reinterpret_cast<Bars*>(smem + kBarOff);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int tile = blockIdx.x, kvh = blockIdx.y, c = blockIdx.z;
+  const int G = p.group;
+  const int QT = BM / G;  // queries per CTA tile
+  const int q0 = p.query_start_loc[c], q1 = p.query_start_loc[c + 1];
+  const int L = q1 - q0;
+  const int ctx = p.context_lens[c];
+  if (L < 0 || L > p.max_chunk_len || ctx < L || ctx > p.max_blocks * 16) {
+    if (threadIdx.x == 0 && tile == 0 && kvh == 0) flag_error(p.dev_err, PA_DEVERR_QUERY_LOC);
+    return;
+  }
+  const int H = ctx - L;
+  const int i0 = tile * QT;
+  if (i0 >= L) return;
+  const int i_end = min(L, i0 + QT);
+  const int n_keys = H + i_end;
+  const int nkt = (n_keys + BN - 1) / BN;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&B->kv_full[s], 128);
+      mbar_init(&B->kv_empty[s], 1);
+      mbar_init(&B->s_full[s], 1);
+      mbar_init(&B->s_empty[s], 128);
+    }
+    mbar_init(&B->p_full, 128);
+    mbar_init(&B->pv_done, 1);
+    mbar_init(&B->done, 1);
+    B->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&B->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  // Q tile -> shared (K-major, swizzled), one row per softmax thread
+  if (tid < BM) {
+    const int r = tid, i = i0 + r / G, g = r % G;
+    const bool valid = i < L;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        reinterpret_cast<const __nv_bfloat16*>(p.q) +
+        ((size_t)(q0 + (valid ? i : 0)) * p.n_q + (size_t)kvh * G + g) * D);
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+      uint4 v = valid ? src[ch] : make_uint4(0, 0, 0, 0);
+      v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                     bf16x2_to_f16x2(v.w));  // the MMAs run in f16
+      *reinterpret_cast<uint4*>(smem + kQOff + op_off(r, ch)) = v;
+    }
+    fence_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = B->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 256;
+
+  if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      // kind::f16: D f32, A and B f16, both K-major, N = 128, M = 128
+      const uint32_t idesc =
+          (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      const uint32_t aQ = sbase + kQOff, aP = sbase + kPOff;
+      bool ok = true;
+      for (int j = 0; j <= nkt && ok; ++j) {
+        if (j < nkt) {
+          const int s = j & 1;
+          ok = wait_or_abort(&B->kv_full[s], (j >> 1) & 1, B, p.dev_err);
+          if (ok && j >= 2) ok = wait_or_abort(&B->s_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bK = sbase + kKOff + s * kOpBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc_mma(tS + s * BN, smem_desc(aQ + off), smem_desc(bK + off), idesc, kk > 0);
+          }
+          tc_commit(&B->s_full[s]);
+        }
+        if (j >= 1) {
+          const int jp = j - 1, s = jp & 1;
+          ok = wait_or_abort(&B->p_full, jp & 1, B, p.dev_err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t bV = sbase + kVOff + s * kOpBytes;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc_mma(tO, smem_desc(aP + off), smem_desc(bV + off), idesc, (jp > 0 || kk > 0));
+          }
+          tc_commit(&B->pv_done);
+          tc_commit(&B->kv_empty[s]);
+        }
+      }
+      // everything issued above has completed before TMEM is released
+      tc_commit(&B->done);
+      mbar_wait(&B->done, 0);
+    }
+  } else if (warp >= kSoftmaxWarps) {
+    // ------------------------------------------------------------ converters
+    const int ct = tid - kSoftmaxWarps * 32;  // 0..127
+    const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
+    const int kv_es = FP8 ? 1 : 2;
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j & 1;
+      bool stop = j >= 2 && !wait_or_abort(&B->kv_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
+      if (conv_bar_or(stop || aborted(B))) break;  // all 128 converters stop together
+      uint8_t* kop = smem + kKOff + s * kOpBytes;
+      uint8_t* vop = smem + kVOff + s * kOpBytes;
+      uint8_t* stg = smem + kStgOff;
+      // each pass covers 128 x 16-byte chunks of stored K and V rows
+      constexpr int kPasses = FP8 ? 8 : 16;
+#pragma unroll 2
+      for (int m = 0; m < kPasses; ++m) {
+        const int blk_in_tile = FP8 ? m : (m >> 1);
+        const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));  // key in block
+        const int cc = FP8 ? (ct & 7) : (ct & 15);  // stored 16-byte chunk within the row
+        const int key_t = blk_in_tile * 16 + kib;    // key within tile
+        const int key = j * BN + key_t;
+        uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
+        if (key < ctx) {
+          int phys = bt[key >> 4];
+          if (phys < 0 || phys >= p.num_blocks) {
+            if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+          } else {
+            const size_t off = (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
+            kraw = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
+            vraw = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
+          }
+        }
+        if constexpr (FP8) {
+          // 16 codes -> 16 f16 = 16-bit chunks 2cc, 2cc+1 (dims 16cc..16cc+15)
+          uint32_t kh[8], vh[8];
+          const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
+          const uint32_t vw[4] = {vraw.x, vraw.y, vraw.z, vraw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
+            kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
+            vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
+            vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
+          }
+          *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
+          *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc + 1)) = make_uint4(kh[4], kh[5], kh[6], kh[7]);
+          *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc)) = make_uint4(vh[0], vh[1], vh[2], vh[3]);
+          *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc + 8)) = make_uint4(vh[4], vh[5], vh[6], vh[7]);
+        } else {
+          *reinterpret_cast<uint4*>(kop + op_off(key_t, cc)) =
+              make_uint4(bf16x2_to_f16x2(kraw.x), bf16x2_to_f16x2(kraw.y),
+                         bf16x2_to_f16x2(kraw.z), bf16x2_to_f16x2(kraw.w));
+          *reinterpret_cast<uint4*>(stg + stg_off(key_t, 8 * cc)) =
+              make_uint4(bf16x2_to_f16x2(vraw.x), bf16x2_to_f16x2(vraw.y),
+                         bf16x2_to_f16x2(vraw.z), bf16x2_to_f16x2(vraw.w));
+        }
+      }
+      conv_bar();
+      // V^T: thread ct builds row d = ct of the transposed tile
+      {
+        const int d = ct;
+#pragma unroll 4
+        for (int kc = 0; kc < BN / 8; ++kc) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k0 = kc * 8 + 2 * e;
+            const uint32_t lo = *reinterpret_cast<const uint16_t*>(stg + stg_off(k0, d));
+            const uint32_t hi = *reinterpret_cast<const uint16_t*>(stg + stg_off(k0 + 1, d));
+            w[e] = lo | (hi << 16);
+          }
+          *reinterpret_cast<uint4*>(vop + op_off(d, kc)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(&B->kv_full[s]);
+      conv_bar();  // staging is reused by the next tile
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = tid;  // row = TMEM lane
+    const int i = i0 + r / G, g = r % G;
+    const bool row_valid = i < L;
+    const int lim = H + i;  // last visible key
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sl = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    float x[BN];
+    bool ok = true;
+    for (int j = 0; j < nkt && ok; ++j) {
+      const int s = j & 1;
+      ok = __all_sync(0xffffffffu, wait_or_abort(&B->s_full[s], (j >> 1) & 1, B, p.dev_err));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + lane_base + s * BN + cc * 32, x + cc * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&B->s_empty[s]);
+      float mx = -INFINITY;
+      const int kbase = j * BN;
+#pragma unroll
+      for (int e = 0; e < BN; ++e) {
+        float v = x[e] * sl;
+        if (row_valid) {
+          if (kbase + e > lim) v = -INFINITY;
+        } else {
+          v = 0.f;  // padding row: finite values, never written out
+        }
+        x[e] = v;
+        mx = fmaxf(mx, v);
+      }
+      const float m_new = fmaxf(m_used, mx);
+      const bool rescale = m_new > m_used + kRescaleLog2;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = exp2f(m_used - m_new);  // 0 on the first tile
+        l *= alpha;
+        m_used = m_new;
+      }
+      float rs = 0.f;
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int e = 0; e < BN; e += 2) {
+        const float a = exp2f(x[e] - m_used), b = exp2f(x[e + 1] - m_used);
+        rs += a + b;
+        pk[e / 2] = pack2<false>(a, b);
+      }
+      l += rs;
+      // P and O are free once the previous tile's O += P V has completed
+      if (j >= 1) {
+        ok = __all_sync(0xffffffffu, wait_or_abort(&B->pv_done, (j - 1) & 1, B, p.dev_err));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+          float o[32];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            tmem_ld32(tO + lane_base + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tO + lane_base + cc * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      uint8_t* prow = smem + kPOff;
+#pragma unroll
+      for (int kc = 0; kc < BN / 8; ++kc)
+        *reinterpret_cast<uint4*>(prow + op_off(r, kc)) =
+            make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&B->p_full);
+    }
+    // epilogue: O / l after the last O += P V
+    if (ok && __all_sync(0xffffffffu, wait_or_abort(&B->pv_done, (nkt - 1) & 1, B, p.dev_err))) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? p.out_mul / l : 0.f;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                           ((size_t)(q0 + (row_valid ? i : 0)) * p.n_q + (size_t)kvh * G + g) * D;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float o[32];
+        tmem_ld32(tO + lane_base + cc * 32, o);
+        tmem_wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack2<true>(o[e] * inv, o[e + 1] * inv);
+            v.y = pack2<true>(o[e + 2] * inv, o[e + 3] * inv);
+            v.z = pack2<true>(o[e + 4] * inv, o[e + 5] * inv);
+            v.w = pack2<true>(o[e + 6] * inv, o[e + 7] * inv);
+            *reinterpret_cast<uint4*>(out + cc * 32 + e) = v;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+template <bool FP8>
+cudaError_t launch_tc(const PrefillParams& p, const void* k_pool, const void* v_pool,
+                      cudaStream_t st) {
+  static cudaError_t attr = cudaFuncSetAttribute(
+      prefill_tc_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  const int QT = BM / p.group;
+  dim3 grid((p.max_chunk_len + QT - 1) / QT, p.n_kv, p.n_chunks);
+  prefill_tc_kernel<FP8><<<grid, kThreads, kSmemBytes, st>>>(p, k_pool, v_pool);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k_pool,
+                           const void* v_pool, cudaStream_t st) {
+  if (p.n_chunks == 0) return cudaSuccess;
+  return kv_dt == PA_FP8_E4M3 ? launch_tc<true>(p, k_pool, v_pool, st)
+                              : launch_tc<false>(p, k_pool, v_pool, st);
+}
+
+}  // namespace pa

@@ -55,7 +55,7 @@ def test_fp8_cache_reduced(B, cuda_device):
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_dtype_group_headdim_grid(B, cuda_device, q_dt, kv_dt, d, G):
     n_kv = 2
-    ctx = np.array([0, 1, 15, 16, 17, 33, 500, 1100], np.int32)
+    ctx = np.array([0, 1, 2, 3, 5, 10, 15, 16, 17, 33, 500, 1100], np.int32)
     spec = W.DecodeSpec("grid", len(ctx), n_kv * G, n_kv, d, q_dt, kv_dt, "fixed", (ctx,),
                         max_ctx=1536, pool_factor=1.3, seed=77 + G + d)
     inp = W.make_decode_inputs(spec, ctx=ctx)

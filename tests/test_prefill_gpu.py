@@ -1,0 +1,101 @@
+"""GPU parity of pa_prefill_paged (tcgen05 chunked prefill) against the oracle.
+
+Small chunks are compared in full with the oracle's causal prefill; the
+full-size mixed-step prefill (2 chunks x 512 queries over a 4096-token paged
+history, fp8 cache) is compared on sampled (query, head) rows, each of which
+the oracle computes as attention over that query's causal prefix.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from pagedattention_paged_kv_pa_b200 import workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B(cuda_device):
+    from pagedattention_paged_kv_pa_b200 import binding
+    return binding
+
+
+def _run(B, inp, dev, max_chunk_len):
+    d = dict(q=inp.q.to(dev), k=inp.k_pool.to(dev), v=inp.v_pool.to(dev),
+             bt=inp.block_tables.to(dev), qsl=inp.query_start_loc.to(dev),
+             cl=inp.context_lens.to(dev))
+    out = torch.full_like(d["q"], float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.pa_prefill_paged(out, d["q"], d["k"], d["v"], d["bt"], d["qsl"], d["cl"], inp.scale,
+                       max_chunk_len, inp.k_scale, inp.v_scale, dev_err=err)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy().astype(np.float64), int(err.item())
+
+
+def _oracle(inp):
+    s = inp.spec
+    return orc.paged_prefill(inp.q.cpu(), inp.k_pool.cpu(), inp.v_pool.cpu(),
+                             inp.block_tables.cpu(), inp.query_start_loc.cpu(),
+                             inp.context_lens.cpu(), inp.scale, s.q_dtype, s.kv_dtype,
+                             inp.k_scale, inp.v_scale)
+
+
+@pytest.mark.parametrize("kv_dt", [W.FP8_E4M3, W.BF16])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_small_chunks_against_oracle(B, cuda_device, kv_dt, G):
+    n_kv = 2
+    spec = W.PrefillSpec("small", 3, 0, 0, n_kv * G, n_kv, 128, W.BF16, kv_dt, extra_blocks=5,
+                         seed=300 + G)
+    chunk_lens = [37, 130, 1]
+    histories = [0, 291, 1000]
+    inp = W.make_prefill_inputs(spec, chunk_lens=chunk_lens, histories=histories)
+    gpu, err = _run(B, inp, cuda_device, max(chunk_lens))
+    assert err == 0
+    P.assert_close(gpu, _oracle(inp), W.BF16, kv_dt, f"prefill G={G} kv={kv_dt}")
+
+
+def test_history_zero_single_chunk_is_causal_self_attention(B, cuda_device):
+    spec = W.PrefillSpec("h0", 1, 200, 0, 32, 8, 128, W.BF16, W.BF16, seed=311)
+    inp = W.make_prefill_inputs(spec)
+    gpu, err = _run(B, inp, cuda_device, 200)
+    assert err == 0
+    P.assert_close(gpu, _oracle(inp), W.BF16, W.BF16, "prefill H=0")
+
+
+def test_chunk_lengths_at_tile_edges(B, cuda_device):
+    # G=4 packs 32 queries per CTA tile; keys come in tiles of 128
+    spec = W.PrefillSpec("edges", 4, 0, 0, 32, 8, 128, W.BF16, W.FP8_E4M3, seed=312)
+    chunk_lens = [32, 33, 64, 31]
+    histories = [128, 127, 129, 16]
+    inp = W.make_prefill_inputs(spec, chunk_lens=chunk_lens, histories=histories)
+    gpu, err = _run(B, inp, cuda_device, 64)
+    assert err == 0
+    P.assert_close(gpu, _oracle(inp), W.BF16, W.FP8_E4M3, "prefill tile edges")
+
+
+def test_mixed_step_prefill_full_size_sampled(B, cuda_device):
+    """2 chunks x 512 queries over a 4096-token history, 32 q / 8 kv heads,
+    fp8 cache, in the launch configuration the mixed-step benchmark uses.
+    Sampled rows: query i of chunk c equals decode attention over the first
+    H + i + 1 keys of that chunk's sequence."""
+    spec = W.MIXED_PREFILL_FP8
+    inp = W.make_prefill_inputs(spec, device=cuda_device)
+    gpu, err = _run(B, inp, cuda_device, spec.chunk_len)
+    assert err == 0
+    rng = np.random.default_rng(1)
+    qsl = inp.query_start_loc.cpu().numpy()
+    cl = inp.context_lens.cpu().numpy()
+    picks = [(c, i) for c in range(spec.n_chunks)
+             for i in sorted(set(rng.choice(spec.chunk_len, 6, replace=False).tolist()) | {0, spec.chunk_len - 1})]
+    rows = [qsl[c] + i for c, i in picks]
+    ctx = np.array([cl[c] - spec.chunk_len + i + 1 for c, i in picks], np.int32)
+    bt = inp.block_tables.cpu()[[c for c, _ in picks]]
+    dec = W.DecodeInputs(W.MIXED_DECODE_FP8.scaled(num_seqs=len(rows)), inp.q[rows], inp.k_pool,
+                         inp.v_pool, bt, torch.from_numpy(ctx), inp.scale, inp.k_scale,
+                         inp.v_scale)
+    sub = P.subset_for_oracle(dec, list(range(len(rows))))
+    ref = P.oracle_decode(sub)
+    P.assert_close(gpu[rows], ref, W.BF16, W.FP8_E4M3, "mixed-step prefill sampled")
+    assert np.isfinite(gpu).all()
