@@ -27,7 +27,7 @@
 // O^T[d][8 heads] += V^T . P^T, each as m16n8k16 warp MMAs with the GQA group
 // as N=8 (fp32 accumulate; with 16-bit caches P enters as a 16-bit value plus
 // its 16-bit rounding residual).  For fp8 caches the E4M3 codes are widened to f16
-// exactly (K in registers, V through a per-warp shared tile) and the
+// exactly in registers after ldmatrix (no shared-memory round trip), and the
 // per-tensor scales are applied to the scores and to the final output.  fp32
 // inputs use a CUDA-core path with fp32 arithmetic throughout.
 #include "pa_device.cuh"
@@ -47,14 +47,12 @@ template <int D, bool FP8>
 struct MmaLayout {
   static constexpr int kTileBytes = 16 * D * (FP8 ? 1 : 2);  // one (block, head) tile
   static constexpr int kStageBytes = 2 * kTileBytes;          // K + V
-  static constexpr int kConvBytes = FP8 ? 16 * D * 2 : 0;     // per-warp f16 V tile
-  static constexpr int kConvOff = kStages * kStageBytes;
-  static constexpr int kIdsOff = kConvOff + kNW * kConvBytes;
+  static constexpr int kIdsOff = kStages * kStageBytes;
   static constexpr int kBarOff = kIdsOff + kPartBlocks * 4;
   static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 1024;  // + align slack
   static constexpr int kMergeFloats = kNW * kMaxGroup * D + 4 * kNW * kMaxGroup + 2 * kMaxGroup;
   static_assert(kMergeFloats * 4 <= kIdsOff, "merge scratch must fit in the ring");
-  static_assert(kStageBytes % 1024 == 0 && kConvBytes % 1024 == 0, "1024-B aligned tiles");
+  static_assert(kStageBytes % 1024 == 0, "1024-B aligned tiles");
 };
 
 template <typename T>
@@ -258,7 +256,6 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     }
     const float sl = p.scale_log2;
     const uint32_t sbase = smem_u32(smem);
-    uint8_t* conv = smem + L::kConvOff + warp * L::kConvBytes;
     const int q4 = lane >> 3;
 
     for (int j = warp; j < nblk; j += kNW) {
@@ -282,17 +279,21 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
             mma_16816<kMmaBf16>(sc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
           }
         } else {
-          const uint8_t* ktp = smem + s * L::kStageBytes;
+          // the fp8 tile read as 16-bit pairs: ldmatrix hands lane (g, t) the 4
+          // codes of dims 4t..4t+3 of a 16-dim step for tokens g and g+8 --
+          // the permuted k pairing the Q fragments were built with
 #pragma unroll
-          for (int kk = 0; kk < KS; ++kk) {
-            const uint32_t o0 = g * D + 16 * kk + 4 * t, o1 = (g + 8) * D + 16 * kk + 4 * t;
-            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(
-                ktp + (D == 128 ? swz128(o0) : swz64(o0)));
-            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(
-                ktp + (D == 128 ? swz128(o1) : swz64(o1)));
-            mma_16816<false>(sc, e4m3x2_to_f16x2(w0 & 0xffffu), e4m3x2_to_f16x2(w1 & 0xffffu),
-                             e4m3x2_to_f16x2(w0 >> 16), e4m3x2_to_f16x2(w1 >> 16), qb[kk][0],
-                             qb[kk][1]);
+          for (int k2 = 0; k2 < KS / 2; ++k2) {
+            const int row = (lane & 7) + ((q4 & 1) << 3);
+            const uint32_t off = row * D + (2 * k2 + (q4 >> 1)) * 16;
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4(kt + (D == 128 ? swz128(off) : swz64(off)), r0, r1, r2, r3);
+            mma_16816<false>(sc, e4m3x2_to_f16x2(r0 & 0xffffu), e4m3x2_to_f16x2(r1 & 0xffffu),
+                             e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16),
+                             qb[2 * k2][0], qb[2 * k2][1]);
+            mma_16816<false>(sc, e4m3x2_to_f16x2(r2 & 0xffffu), e4m3x2_to_f16x2(r3 & 0xffffu),
+                             e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16),
+                             qb[2 * k2 + 1][0], qb[2 * k2 + 1][1]);
           }
         }
         // ---- online softmax (log2 domain); lane holds tokens g, g+8 of heads 2t, 2t+1
@@ -312,12 +313,14 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
         l1 = l1 * c1 + (p1 + p3);
         m0 = n0;
         m1 = n1;
+        if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {  // a running max grew
 #pragma unroll
-        for (int i = 0; i < KS; ++i) {
-          o[i][0] *= c0;
-          o[i][1] *= c1;
-          o[i][2] *= c0;
-          o[i][3] *= c1;
+          for (int i = 0; i < KS; ++i) {
+            o[i][0] *= c0;
+            o[i][1] *= c1;
+            o[i][2] *= c0;
+            o[i][3] *= c1;
+          }
         }
         // P^T as the B operand: transpose the two 8x8 (token x head) halves.
         // With 16-bit caches P is split into a rounded part and its rounding
@@ -332,63 +335,51 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
           pl0 = movmatrix_t(pack2<kMmaBf16>(p0 - h01.x, p1 - h01.y));
           pl1 = movmatrix_t(pack2<kMmaBf16>(p2 - h23.x, p3 - h23.y));
         }
-        // ---- V^T tiles (A operand), O^T += V^T . P^T
-        uint32_t vbase;
+        // ---- V^T tiles (A operand), O^T += V^T . P^T; tokens past the context
+        // are masked out of V (their bytes are not part of the sequence)
         uint32_t mk01 = 0xffffffffu, mk23 = 0xffffffffu;
-        if constexpr (FP8) {
-          // widen the fp8 V tile to f16 in this warp's tile, zeroing rows
-          // past the context (their bytes are not part of the sequence)
-          const uint8_t* vsrc = smem + s * L::kStageBytes + L::kTileBytes;
-          constexpr int CH = D / 16;
-          __syncwarp();
-#pragma unroll
-          for (int ci = lane; ci < 16 * CH; ci += 32) {
-            const int r = ci / CH, pc = ci % CH;
-            const int lc = (D == 128) ? (pc ^ (r & 7)) : (pc ^ ((r >> 1) & 3));
-            uint4 raw = *reinterpret_cast<const uint4*>(vsrc + r * D + pc * 16);
-            uint32_t h[8];
-            if (r < valid) {
-              h[0] = e4m3x2_to_f16x2(raw.x & 0xffffu);
-              h[1] = e4m3x2_to_f16x2(raw.x >> 16);
-              h[2] = e4m3x2_to_f16x2(raw.y & 0xffffu);
-              h[3] = e4m3x2_to_f16x2(raw.y >> 16);
-              h[4] = e4m3x2_to_f16x2(raw.z & 0xffffu);
-              h[5] = e4m3x2_to_f16x2(raw.z >> 16);
-              h[6] = e4m3x2_to_f16x2(raw.w & 0xffffu);
-              h[7] = e4m3x2_to_f16x2(raw.w >> 16);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) h[e] = 0u;
-            }
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-              const int C = 2 * lc + c2;
-              *reinterpret_cast<uint4*>(conv + swz128((C >> 3) * 2048 + r * 128 + (C & 7) * 16)) =
-                  make_uint4(h[4 * c2], h[4 * c2 + 1], h[4 * c2 + 2], h[4 * c2 + 3]);
-            }
-          }
-          __syncwarp();
-          vbase = smem_u32(conv);
-        } else {
-          vbase = kt + L::kTileBytes;
-          if (valid < 16) {
-            mk01 = ((2 * t < valid) ? 0x0000ffffu : 0u) | ((2 * t + 1 < valid) ? 0xffff0000u : 0u);
-            mk23 = ((2 * t + 8 < valid) ? 0x0000ffffu : 0u) |
-                   ((2 * t + 9 < valid) ? 0xffff0000u : 0u);
-          }
+        if (valid < 16) {
+          mk01 = ((2 * t < valid) ? 0x0000ffffu : 0u) | ((2 * t + 1 < valid) ? 0xffff0000u : 0u);
+          mk23 = ((2 * t + 8 < valid) ? 0x0000ffffu : 0u) |
+                 ((2 * t + 9 < valid) ? 0xffff0000u : 0u);
         }
+        if constexpr (!FP8) {
+          const uint32_t vbase = kt + L::kTileBytes;
 #pragma unroll
-        for (int i = 0; i < KS; ++i) {
-          const int row = (lane & 7) + ((q4 >> 1) << 3);
-          const int C = 2 * i + (q4 & 1);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(vbase + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2, a3);
-          a0 &= mk01;
-          a1 &= mk01;
-          a2 &= mk23;
-          a3 &= mk23;
-          mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pb0, pb1);
-          if constexpr (!FP8) mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pl0, pl1);
+          for (int i = 0; i < KS; ++i) {
+            const int row = (lane & 7) + ((q4 >> 1) << 3);
+            const int C = 2 * i + (q4 & 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vbase + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2, a3);
+            a0 &= mk01;
+            a1 &= mk01;
+            a2 &= mk23;
+            a3 &= mk23;
+            mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pb0, pb1);
+            mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pl0, pl1);
+          }
+        } else {
+          // the fp8 V tile read as 16-bit pairs with ldmatrix.trans: a lane gets
+          // the codes of dims (2g, 2g+1) of a 16-dim step for tokens (2t, 2t+1);
+          // byte permutes split them into one V^T row per dim.  MMA row g holds
+          // dim 16i+2g and row g+8 dim 16i+2g+1 (undone when O is written out).
+          const uint32_t vbase = kt + L::kTileBytes;
+#pragma unroll
+          for (int i2 = 0; i2 < KS / 2; ++i2) {
+            const int row = (lane & 7) + ((q4 & 1) << 3);
+            const uint32_t off = row * D + (2 * i2 + (q4 >> 1)) * 16;
+            uint32_t r[4];
+            ldsm_x4_t(vbase + (D == 128 ? swz128(off) : swz64(off)), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t lo = r[2 * h], hi = r[2 * h + 1];  // tokens 0-7 / 8-15
+              const uint32_t a0 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020u)) & mk01;
+              const uint32_t a1 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031u)) & mk01;
+              const uint32_t a2 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020u)) & mk23;
+              const uint32_t a3 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031u)) & mk23;
+              mma_16816<false>(o[2 * i2 + h], a0, a1, a2, a3, pb0, pb1);
+            }
+          }
         }
       }
       __syncwarp();
@@ -411,12 +402,15 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   float* Ms = Ls + 8;
   if (warp < kNW) {
     float* mw = mo + warp * 8 * D;
+    // O^T row g / g+8 of m-tile i is dim 16i+g / 16i+g+8 (16-bit caches) or
+    // dim 16i+2g / 16i+2g+1 (fp8 caches)
+    const int d_lo = FP8 ? 2 * g : g, d_hi = FP8 ? 2 * g + 1 : g + 8;
 #pragma unroll
     for (int i = 0; i < KS; ++i) {
-      mw[(2 * t) * D + 16 * i + g] = o[i][0];
-      mw[(2 * t + 1) * D + 16 * i + g] = o[i][1];
-      mw[(2 * t) * D + 16 * i + g + 8] = o[i][2];
-      mw[(2 * t + 1) * D + 16 * i + g + 8] = o[i][3];
+      mw[(2 * t) * D + 16 * i + d_lo] = o[i][0];
+      mw[(2 * t + 1) * D + 16 * i + d_lo] = o[i][1];
+      mw[(2 * t) * D + 16 * i + d_hi] = o[i][2];
+      mw[(2 * t + 1) * D + 16 * i + d_hi] = o[i][3];
     }
     if (g == 0) {
       mm[warp * 8 + 2 * t] = m0;

@@ -289,54 +289,79 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kv_es = FP8 ? 1 : 2;
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1;
-      bool stop = j >= 2 && !wait_or_abort(&B->kv_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
-      if (conv_bar_or(stop || aborted(B))) break;  // all 128 converters stop together
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + s * kOpBytes;
       uint8_t* stg = smem + kStgOff;
-      // each pass covers 128 x 16-byte chunks of stored K and V rows
+      // each pass covers 128 x 16-byte chunks of stored K and V rows; the loads
+      // of 8 passes are issued together, then converted and stored.  The first
+      // group's loads go out before waiting for the stage to be released, so
+      // their latency overlaps the tensor-core work still reading the stage.
       constexpr int kPasses = FP8 ? 8 : 16;
-#pragma unroll 2
-      for (int m = 0; m < kPasses; ++m) {
-        const int blk_in_tile = FP8 ? m : (m >> 1);
-        const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));  // key in block
-        const int cc = FP8 ? (ct & 7) : (ct & 15);  // stored 16-byte chunk within the row
-        const int key_t = blk_in_tile * 16 + kib;    // key within tile
-        const int key = j * BN + key_t;
-        uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
-        if (key < ctx) {
-          int phys = bt[key >> 4];
-          if (phys < 0 || phys >= p.num_blocks) {
-            if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
-          } else {
-            const size_t off = (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
-            kraw = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
-            vraw = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
+      constexpr int kGroup = 8;
+#pragma unroll
+      for (int g0 = 0; g0 < kPasses; g0 += kGroup) {
+        uint4 kr[kGroup], vr[kGroup];
+#pragma unroll
+        for (int u = 0; u < kGroup; ++u) {
+          const int m = g0 + u;
+          const int blk_in_tile = FP8 ? m : (m >> 1);
+          const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));  // key in block
+          const int cc = FP8 ? (ct & 7) : (ct & 15);  // stored 16-byte chunk in the row
+          const int key = j * BN + blk_in_tile * 16 + kib;
+          kr[u] = make_uint4(0, 0, 0, 0);
+          vr[u] = make_uint4(0, 0, 0, 0);
+          if (key < ctx) {
+            const int phys = __ldg(&bt[key >> 4]);
+            if (phys < 0 || phys >= p.num_blocks) {
+              if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+            } else {
+              const size_t off =
+                  (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
+              kr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
+              vr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
+            }
           }
         }
-        if constexpr (FP8) {
-          // 16 codes -> 16 f16 = 16-bit chunks 2cc, 2cc+1 (dims 16cc..16cc+15)
-          uint32_t kh[8], vh[8];
-          const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
-          const uint32_t vw[4] = {vraw.x, vraw.y, vraw.z, vraw.w};
+        if (g0 == 0) {
+          const bool stop =
+              j >= 2 && !wait_or_abort(&B->kv_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
+          if (conv_bar_or(stop || aborted(B))) goto conv_done;  // all converters stop together
+        }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
-            kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
-            vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
-            vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
+        for (int u = 0; u < kGroup; ++u) {
+          const int m = g0 + u;
+          const int blk_in_tile = FP8 ? m : (m >> 1);
+          const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));
+          const int cc = FP8 ? (ct & 7) : (ct & 15);
+          const int key_t = blk_in_tile * 16 + kib;  // key within tile
+          if constexpr (FP8) {
+            // 16 codes -> 16 f16 = 16-bit chunks 2cc, 2cc+1 (dims 16cc..16cc+15)
+            uint32_t kh[8], vh[8];
+            const uint32_t kw[4] = {kr[u].x, kr[u].y, kr[u].z, kr[u].w};
+            const uint32_t vw[4] = {vr[u].x, vr[u].y, vr[u].z, vr[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
+              kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
+              vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
+              vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
+            }
+            *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc)) =
+                make_uint4(kh[0], kh[1], kh[2], kh[3]);
+            *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc + 1)) =
+                make_uint4(kh[4], kh[5], kh[6], kh[7]);
+            *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc)) =
+                make_uint4(vh[0], vh[1], vh[2], vh[3]);
+            *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc + 8)) =
+                make_uint4(vh[4], vh[5], vh[6], vh[7]);
+          } else {
+            *reinterpret_cast<uint4*>(kop + op_off(key_t, cc)) =
+                make_uint4(bf16x2_to_f16x2(kr[u].x), bf16x2_to_f16x2(kr[u].y),
+                           bf16x2_to_f16x2(kr[u].z), bf16x2_to_f16x2(kr[u].w));
+            *reinterpret_cast<uint4*>(stg + stg_off(key_t, 8 * cc)) =
+                make_uint4(bf16x2_to_f16x2(vr[u].x), bf16x2_to_f16x2(vr[u].y),
+                           bf16x2_to_f16x2(vr[u].z), bf16x2_to_f16x2(vr[u].w));
           }
-          *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc)) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-          *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc + 1)) = make_uint4(kh[4], kh[5], kh[6], kh[7]);
-          *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc)) = make_uint4(vh[0], vh[1], vh[2], vh[3]);
-          *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc + 8)) = make_uint4(vh[4], vh[5], vh[6], vh[7]);
-        } else {
-          *reinterpret_cast<uint4*>(kop + op_off(key_t, cc)) =
-              make_uint4(bf16x2_to_f16x2(kraw.x), bf16x2_to_f16x2(kraw.y),
-                         bf16x2_to_f16x2(kraw.z), bf16x2_to_f16x2(kraw.w));
-          *reinterpret_cast<uint4*>(stg + stg_off(key_t, 8 * cc)) =
-              make_uint4(bf16x2_to_f16x2(vraw.x), bf16x2_to_f16x2(vraw.y),
-                         bf16x2_to_f16x2(vraw.z), bf16x2_to_f16x2(vraw.w));
         }
       }
       conv_bar();
@@ -360,6 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&B->kv_full[s]);
       conv_bar();  // staging is reused by the next tile
     }
+  conv_done:;
   } else {
     // ------------------------------------------------------------ softmax
     const int r = tid;  // row = TMEM lane
