@@ -506,7 +506,8 @@ def run_mixed(args, rank, world, local):
                           "peak_tflops": tflops_peak, "frac": round(pre_tflops / tflops_peak, 4),
                           "peak_source": tsrc, "includes": "slot write + prefill kernel"},
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(dec_gbs / peak, 4), "traffic": None,
+                     "frac": round(dec_gbs / peak, 4),
+                     "traffic": traffic_from_profile("mixed_step_fp8_decode"),
                      "kernel": "decode_mma_kernel (fp8 cache)"},
         "gpu_launches": 5 * K,
         "clocks": clocks,

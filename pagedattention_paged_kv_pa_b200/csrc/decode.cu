@@ -30,6 +30,8 @@
 // exactly in registers after ldmatrix (no shared-memory round trip), and the
 // per-tensor scales are applied to the scores and to the final output.  fp32
 // inputs use a CUDA-core path with fp32 arithmetic throughout.
+#include <type_traits>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -343,44 +345,61 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
           mk23 = ((2 * t + 8 < valid) ? 0x0000ffffu : 0u) |
                  ((2 * t + 9 < valid) ? 0xffff0000u : 0u);
         }
-        if constexpr (!FP8) {
-          const uint32_t vbase = kt + L::kTileBytes;
+        // the masks are applied only in a partition's partial last block
+        auto pv = [&](auto masked) {
+          constexpr bool kMask = decltype(masked)::value;
+          if constexpr (!FP8) {
+            const uint32_t vbase = kt + L::kTileBytes;
 #pragma unroll
-          for (int i = 0; i < KS; ++i) {
-            const int row = (lane & 7) + ((q4 >> 1) << 3);
-            const int C = 2 * i + (q4 & 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(vbase + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2, a3);
-            a0 &= mk01;
-            a1 &= mk01;
-            a2 &= mk23;
-            a3 &= mk23;
-            mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pb0, pb1);
-            mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pl0, pl1);
-          }
-        } else {
-          // the fp8 V tile read as 16-bit pairs with ldmatrix.trans: a lane gets
-          // the codes of dims (2g, 2g+1) of a 16-dim step for tokens (2t, 2t+1);
-          // byte permutes split them into one V^T row per dim.  MMA row g holds
-          // dim 16i+2g and row g+8 dim 16i+2g+1 (undone when O is written out).
-          const uint32_t vbase = kt + L::kTileBytes;
+            for (int i = 0; i < KS; ++i) {
+              const int row = (lane & 7) + ((q4 >> 1) << 3);
+              const int C = 2 * i + (q4 & 1);
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_t(vbase + swz128((C >> 3) * 2048 + row * 128 + (C & 7) * 16), a0, a1, a2,
+                        a3);
+              if constexpr (kMask) {
+                a0 &= mk01;
+                a1 &= mk01;
+                a2 &= mk23;
+                a3 &= mk23;
+              }
+              mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pb0, pb1);
+              mma_16816<kMmaBf16>(o[i], a0, a1, a2, a3, pl0, pl1);
+            }
+          } else {
+            // the fp8 V tile read as 16-bit pairs with ldmatrix.trans: a lane gets
+            // the codes of dims (2g, 2g+1) of a 16-dim step for tokens (2t, 2t+1);
+            // byte permutes split them into one V^T row per dim.  MMA row g holds
+            // dim 16i+2g and row g+8 dim 16i+2g+1 (undone when O is written out).
+            const uint32_t vbase = kt + L::kTileBytes;
 #pragma unroll
-          for (int i2 = 0; i2 < KS / 2; ++i2) {
-            const int row = (lane & 7) + ((q4 & 1) << 3);
-            const uint32_t off = row * D + (2 * i2 + (q4 >> 1)) * 16;
-            uint32_t r[4];
-            ldsm_x4_t(vbase + (D == 128 ? swz128(off) : swz64(off)), r[0], r[1], r[2], r[3]);
+            for (int i2 = 0; i2 < KS / 2; ++i2) {
+              const int row = (lane & 7) + ((q4 & 1) << 3);
+              const uint32_t off = row * D + (2 * i2 + (q4 >> 1)) * 16;
+              uint32_t r[4];
+              ldsm_x4_t(vbase + (D == 128 ? swz128(off) : swz64(off)), r[0], r[1], r[2], r[3]);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t lo = r[2 * h], hi = r[2 * h + 1];  // tokens 0-7 / 8-15
-              const uint32_t a0 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020u)) & mk01;
-              const uint32_t a1 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031u)) & mk01;
-              const uint32_t a2 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020u)) & mk23;
-              const uint32_t a3 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031u)) & mk23;
-              mma_16816<false>(o[2 * i2 + h], a0, a1, a2, a3, pb0, pb1);
+              for (int h = 0; h < 2; ++h) {
+                const uint32_t lo = r[2 * h], hi = r[2 * h + 1];  // tokens 0-7 / 8-15
+                uint32_t a0 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020u));
+                uint32_t a1 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031u));
+                uint32_t a2 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020u));
+                uint32_t a3 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031u));
+                if constexpr (kMask) {
+                  a0 &= mk01;
+                  a1 &= mk01;
+                  a2 &= mk23;
+                  a3 &= mk23;
+                }
+                mma_16816<false>(o[2 * i2 + h], a0, a1, a2, a3, pb0, pb1);
+              }
             }
           }
-        }
+        };
+        if (valid < 16)
+          pv(std::true_type{});
+        else
+          pv(std::false_type{});
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);

@@ -12,8 +12,8 @@
 // group).  Keys are processed in tiles of 128 (8 blocks of 16 from the block
 // table).  Warp roles (288 threads):
 //   warps 0-3  softmax: thread r owns row r = TMEM lane r; reads S from TMEM,
-//              masks, keeps an online max/sum, writes P (16-bit) to shared
-//              memory, rescales the TMEM output when its max grew by more
+//              masks, keeps an online max/sum, writes P (f16) to shared
+//              memory, rescales the TMEM output only when its max grew by more
 //              than 2^8, and writes the normalised output at the end;
 //   warps 4-7  K/V converters: load a tile's K and V rows through the block
 //              table with coalesced 16-byte loads, widen fp8 codes exactly to
@@ -30,6 +30,8 @@
 // this tile's softmax; K/V operands are double buffered.  All waits are
 // bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA drains its
 // tensor-core work and frees its TMEM before returning.
+#include <type_traits>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -138,6 +140,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+// 2^x with the hardware approximation (relative error far below f16's 2^-11;
+// results below 2^-126 flush to zero, which P can afford)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -287,27 +296,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ct = tid - kSoftmaxWarps * 32;  // 0..127
     const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
     const int kv_es = FP8 ? 1 : 2;
+    // K- and V-tile writers shared by both paths
+    auto write_v_transposed = [&](uint8_t* vop, const uint8_t* stg) {
+      // V^T: thread ct builds rows 2dp and 2dp+1 of the transposed tile for one
+      // half of the keys, reading both dims of a key with one 32-bit load
+      const int dp = ct & 63, kh = ct >> 6;
+#pragma unroll 2
+      for (int kc = kh * 8; kc < kh * 8 + 8; ++kc) {
+        uint32_t wa[4], wb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int k0 = kc * 8 + 2 * e;
+          const uint32_t u0 = *reinterpret_cast<const uint32_t*>(stg + stg_off(k0, 2 * dp));
+          const uint32_t u1 = *reinterpret_cast<const uint32_t*>(stg + stg_off(k0 + 1, 2 * dp));
+          wa[e] = __byte_perm(u0, u1, 0x5410u);  // (key k0, key k0+1) of dim 2dp
+          wb[e] = __byte_perm(u0, u1, 0x7632u);  // same keys of dim 2dp+1
+        }
+        *reinterpret_cast<uint4*>(vop + op_off(2 * dp, kc)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        *reinterpret_cast<uint4*>(vop + op_off(2 * dp + 1, kc)) =
+            make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      }
+    };
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + s * kOpBytes;
       uint8_t* stg = smem + kStgOff;
-      // each pass covers 128 x 16-byte chunks of stored K and V rows; the loads
-      // of 8 passes are issued together, then converted and stored.  The first
-      // group's loads go out before waiting for the stage to be released, so
-      // their latency overlaps the tensor-core work still reading the stage.
+      // Each pass covers 128 x 16-byte chunks of stored K and V rows: for fp8,
+      // pass m is block m of the tile (thread ct: key ct/8, chunk ct%8); for
+      // bf16, pass m is half of block m/2 (key 8(m%2) + ct/16, chunk ct%16).
+      // The loads of 8 passes go out together; the first group's before the
+      // stage is released, so their latency overlaps the tensor-core work
+      // still reading it.
       constexpr int kPasses = FP8 ? 8 : 16;
-      constexpr int kGroup = 8;
 #pragma unroll
-      for (int g0 = 0; g0 < kPasses; g0 += kGroup) {
-        uint4 kr[kGroup], vr[kGroup];
+      for (int g0 = 0; g0 < kPasses; g0 += 8) {
+        uint4 kr[8], vr[8];
 #pragma unroll
-        for (int u = 0; u < kGroup; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int m = g0 + u;
-          const int blk_in_tile = FP8 ? m : (m >> 1);
           const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));  // key in block
-          const int cc = FP8 ? (ct & 7) : (ct & 15);  // stored 16-byte chunk in the row
-          const int key = j * BN + blk_in_tile * 16 + kib;
+          const int cc = FP8 ? (ct & 7) : (ct & 15);  // 16-byte chunk in the row
+          const int key = j * BN + (FP8 ? m : (m >> 1)) * 16 + kib;
           kr[u] = make_uint4(0, 0, 0, 0);
           vr[u] = make_uint4(0, 0, 0, 0);
           if (key < ctx) {
@@ -315,8 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (phys < 0 || phys >= p.num_blocks) {
               if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
             } else {
-              const size_t off =
-                  (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
+              const size_t off = (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
               kr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
               vr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
             }
@@ -328,12 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (conv_bar_or(stop || aborted(B))) goto conv_done;  // all converters stop together
         }
 #pragma unroll
-        for (int u = 0; u < kGroup; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int m = g0 + u;
-          const int blk_in_tile = FP8 ? m : (m >> 1);
           const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));
           const int cc = FP8 ? (ct & 7) : (ct & 15);
-          const int key_t = blk_in_tile * 16 + kib;  // key within tile
+          const int key_t = (FP8 ? m : (m >> 1)) * 16 + kib;  // key within tile
           if constexpr (FP8) {
             // 16 codes -> 16 f16 = 16-bit chunks 2cc, 2cc+1 (dims 16cc..16cc+15)
             uint32_t kh[8], vh[8];
@@ -365,22 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       conv_bar();
-      // V^T: thread ct builds row d = ct of the transposed tile
-      {
-        const int d = ct;
-#pragma unroll 4
-        for (int kc = 0; kc < BN / 8; ++kc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k0 = kc * 8 + 2 * e;
-            const uint32_t lo = *reinterpret_cast<const uint16_t*>(stg + stg_off(k0, d));
-            const uint32_t hi = *reinterpret_cast<const uint16_t*>(stg + stg_off(k0 + 1, d));
-            w[e] = lo | (hi << 16);
-          }
-          *reinterpret_cast<uint4*>(vop + op_off(d, kc)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
+      write_v_transposed(vop, stg);
       fence_async_smem();
       mbar_arrive(&B->kv_full[s]);
       conv_bar();  // staging is reused by the next tile
@@ -395,31 +408,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float sl = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
-    float x[BN];
     bool ok = true;
     for (int j = 0; j < nkt && ok; ++j) {
       const int s = j & 1;
       ok = __all_sync(0xffffffffu, wait_or_abort(&B->s_full[s], (j >> 1) & 1, B, p.dev_err));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + lane_base + s * BN + cc * 32, x + cc * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&B->s_empty[s]);
-      float mx = -INFINITY;
       const int kbase = j * BN;
+      const uint32_t tSrow = tS + lane_base + s * BN;
+      // a tile every key of which is visible to every row of this warp needs no
+      // mask: its max is taken on the raw scores (the scale is positive)
+      const bool full = __all_sync(0xffffffffu, row_valid && kbase + BN - 1 <= lim) && sl > 0.f;
+      // pass 1: the row's max over this tile, 32 columns at a time
+      float mx = -INFINITY;
+      if (full) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float x[32];
+          tmem_ld32(tSrow + cc * 32, x);
+          tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < BN; ++e) {
-        float v = x[e] * sl;
-        if (row_valid) {
-          if (kbase + e > lim) v = -INFINITY;
-        } else {
-          v = 0.f;  // padding row: finite values, never written out
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, x[e]);
         }
-        x[e] = v;
-        mx = fmaxf(mx, v);
+        mx *= sl;
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float x[32];
+          tmem_ld32(tSrow + cc * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const bool vis = !row_valid || (kbase + cc * 32 + e <= lim);
+            mx = fmaxf(mx, vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
+          }
+        }
       }
+      // O and l are rescaled lazily: only when the max grew by more than 2^8
       const float m_new = fmaxf(m_used, mx);
       const bool rescale = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
@@ -428,14 +453,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         m_used = m_new;
       }
+      // pass 2: P = 2^(s*scale - m) as f16, kept in registers until the P
+      // buffer is free
       float rs = 0.f;
       uint32_t pk[BN / 2];
+      const float neg_m = -m_used;
+      if (full) {
 #pragma unroll
-      for (int e = 0; e < BN; e += 2) {
-        const float a = exp2f(x[e] - m_used), b = exp2f(x[e + 1] - m_used);
-        rs += a + b;
-        pk[e / 2] = pack2<false>(a, b);
+        for (int cc = 0; cc < 4; ++cc) {
+          float x[32];
+          tmem_ld32(tSrow + cc * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float a = fast_exp2(fmaf(x[e], sl, neg_m));
+            const float bb = fast_exp2(fmaf(x[e + 1], sl, neg_m));
+            rs += a + bb;
+            pk[cc * 16 + e / 2] = pack2<false>(a, bb);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float x[32];
+          tmem_ld32(tSrow + cc * 32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int k0 = kbase + cc * 32 + e;
+            const float v0 = row_valid ? (k0 <= lim ? x[e] * sl : -INFINITY) : 0.f;
+            const float v1 = row_valid ? (k0 + 1 <= lim ? x[e + 1] * sl : -INFINITY) : 0.f;
+            const float a = fast_exp2(v0 + neg_m), bb = fast_exp2(v1 + neg_m);
+            rs += a + bb;
+            pk[cc * 16 + e / 2] = pack2<false>(a, bb);
+          }
+        }
       }
+      tc_fence_before();
+      mbar_arrive(&B->s_empty[s]);  // S buffer s may be overwritten by S(j+2)
       l += rs;
       // P and O are free once the previous tile's O += P V has completed
       if (j >= 1) {
@@ -443,9 +498,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
-          float o[32];
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
+            float o[32];
             tmem_ld32(tO + lane_base + cc * 32, o);
             tmem_wait_ld();
 #pragma unroll
