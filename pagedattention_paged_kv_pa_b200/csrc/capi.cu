@@ -13,6 +13,9 @@ using pa::DecodeParams;
 using pa::ReduceParams;
 
 constexpr float kLog2e = 1.4426950408889634f;
+// The decode kernel widens fp8 V codes to f16 as code x 2^-8; the output
+// scale undoes it (exact: a power of two).
+constexpr float kFp8VUnscale = 256.f;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -205,7 +208,7 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
                       : nullptr;
   p.dev_err = dev_err;
   p.scale_log2 = scale * kLog2e * (fp8 ? k_scale : 1.f);
-  p.out_mul = fp8 ? v_scale : 1.f;
+  p.out_mul = fp8 ? v_scale * kFp8VUnscale : 1.f;
   p.n_q = n_q_heads;
   p.n_kv = n_kv_heads;
   p.group = n_q_heads / n_kv_heads;
@@ -243,7 +246,7 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
   r.ws_o = static_cast<const float*>(workspace);
   r.ws_ml = reinterpret_cast<const float2*>(static_cast<const char*>(workspace) +
                                             ((ws_o_bytes(s) + 255) & ~size_t(255)));
-  r.out_mul = kv_dtype == PA_FP8_E4M3 ? v_scale : 1.f;
+  r.out_mul = kv_dtype == PA_FP8_E4M3 ? v_scale * kFp8VUnscale : 1.f;
   r.n_q = n_q_heads;
   r.num_seqs = num_seqs;
   r.max_blocks = max_blocks_per_seq;

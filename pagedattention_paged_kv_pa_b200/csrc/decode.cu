@@ -381,10 +381,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const uint32_t lo = r[2 * h], hi = r[2 * h + 1];  // tokens 0-7 / 8-15
-                uint32_t a0 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020u));
-                uint32_t a1 = e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031u));
-                uint32_t a2 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020u));
-                uint32_t a3 = e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031u));
+                // widened on the integer pipe (x 2^-8, folded into the output
+                // scale) so that K's hardware conversions have the
+                // conversion pipe to themselves
+                uint32_t a0 = e4m3x2_to_f16x2_div256(lo, 0x4240u);
+                uint32_t a1 = e4m3x2_to_f16x2_div256(lo, 0x4341u);
+                uint32_t a2 = e4m3x2_to_f16x2_div256(hi, 0x4240u);
+                uint32_t a3 = e4m3x2_to_f16x2_div256(hi, 0x4341u);
                 if constexpr (kMask) {
                   a0 &= mk01;
                   a1 &= mk01;

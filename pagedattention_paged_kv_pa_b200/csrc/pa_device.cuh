@@ -189,6 +189,17 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
   return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
+// Two E4M3 codes, picked out of w by the byte selector (result bytes 0 and 2),
+// as an f16x2 holding code x 2^-8, exactly, using integer ops only: with the
+// code s.eeee.mmm in the low byte of a 16-bit lane, (b + (b & 0x80)) << 7
+// puts eeee.mmm into f16's exponent/mantissa fields (bias 15 instead of 7,
+// hence 2^-8; subnormal codes land on f16 subnormals) and the add carries the
+// sign from bit 14 into bit 15.  E4M3's NaN code maps to a finite value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_div256(uint32_t w, uint32_t sel) {
+  const uint32_t y = __byte_perm(w, 0u, sel);  // [b_i, 0, b_j, 0]
+  return (y + (y & 0x00800080u)) << 7;
+}
+
 __device__ __forceinline__ float warp_max_xor(float v, int lo_mask) {
   for (int m = 16; m >= lo_mask; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
   return v;

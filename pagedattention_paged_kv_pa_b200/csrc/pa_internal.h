@@ -25,7 +25,7 @@ struct DecodeParams {
   float2* ws_ml;  // [num_seqs][n_q][n_parts_max] (log2-domain max, sum)
   int32_t* dev_err;
   float scale_log2;  // scale * log2(e) (* k_scale for fp8 caches)
-  float out_mul;     // v_scale for fp8 caches, else 1
+  float out_mul;     // fp8 caches: v_scale x 256 (V is widened as code x 2^-8); else 1
   int n_q, n_kv, group, num_seqs, max_blocks, num_blocks, n_parts_max;
 };
 
