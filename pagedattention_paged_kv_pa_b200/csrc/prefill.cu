@@ -317,11 +317,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             make_uint4(wb[0], wb[1], wb[2], wb[3]);
       }
     };
+    // block ids of a tile's 8 blocks (-1 past the context); the next tile's
+    // are loaded a tile ahead so the K/V loads never wait on the block table
+    auto load_ids = [&](int j, int (&ids)[8]) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int blk = j * 8 + m;
+        ids[m] = (blk * 16 < ctx) ? __ldg(&bt[blk]) : -1;
+      }
+    };
+    int id_cur[8], id_nxt[8];
+    load_ids(0, id_cur);
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + s * kOpBytes;
       uint8_t* stg = smem + kStgOff;
+      if (j + 1 < nkt) load_ids(j + 1, id_nxt);
       // Each pass covers 128 x 16-byte chunks of stored K and V rows: for fp8,
       // pass m is block m of the tile (thread ct: key ct/8, chunk ct%8); for
       // bf16, pass m is half of block m/2 (key 8(m%2) + ct/16, chunk ct%16).
@@ -341,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           kr[u] = make_uint4(0, 0, 0, 0);
           vr[u] = make_uint4(0, 0, 0, 0);
           if (key < ctx) {
-            const int phys = __ldg(&bt[key >> 4]);
+            const int phys = id_cur[FP8 ? m : (m >> 1)];
             if (phys < 0 || phys >= p.num_blocks) {
               if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
             } else {
@@ -397,6 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       mbar_arrive(&B->kv_full[s]);
       conv_bar();  // staging is reused by the next tile
+#pragma unroll
+      for (int m = 0; m < 8; ++m) id_cur[m] = id_nxt[m];
     }
   conv_done:;
   } else {
@@ -423,12 +437,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float mx = -INFINITY;
       if (full) {
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float x[32];
+        for (int cc = 0; cc < 4; cc += 2) {  // two TMEM loads in flight
+          float x[64];
           tmem_ld32(tSrow + cc * 32, x);
+          tmem_ld32(tSrow + cc * 32 + 32, x + 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, x[e]);
+          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, x[e]);
         }
         mx *= sl;
       } else {
