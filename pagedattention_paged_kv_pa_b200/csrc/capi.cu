@@ -13,8 +13,8 @@ using pa::DecodeParams;
 using pa::ReduceParams;
 
 constexpr float kLog2e = 1.4426950408889634f;
-// The decode kernel widens fp8 V codes to f16 as code x 2^-8; the output
-// scale undoes it (exact: a power of two).
+// The decode and prefill kernels widen fp8 V codes to f16 as code x 2^-8; the
+// output scale undoes it (exact: a power of two).
 constexpr float kFp8VUnscale = 256.f;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -305,7 +305,7 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
   p.context_lens = context_lens;
   p.dev_err = dev_err;
   p.scale_log2 = scale * kLog2e * (fp8 ? k_scale : 1.f);
-  p.out_mul = fp8 ? v_scale : 1.f;
+  p.out_mul = fp8 ? v_scale * kFp8VUnscale : 1.f;  // fp8 V is widened as code x 2^-8
   p.n_q = n_q_heads;
   p.n_kv = n_kv_heads;
   p.group = G;

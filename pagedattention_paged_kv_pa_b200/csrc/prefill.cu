@@ -17,11 +17,17 @@
 //              than 2^8, and writes the normalised output at the end;
 //   warps 4-7  K/V converters: load a tile's K and V rows through the block
 //              table with coalesced 16-byte loads, widen fp8 codes exactly to
-//              f16 (bf16 values are converted to f16), write K in the K-major
-//              128-byte-swizzled layout the MMA reads and V transposed (V^T,
-//              also K-major);
+//              f16 (K on the conversion pipe; V on the integer pipe as
+//              code x 2^-8, folded into the output scale; bf16 values are
+//              converted to f16) and write both as [key][d] rows in the
+//              128-byte-swizzled layout: K-major for K, MN-major for V, so V
+//              needs no transpose;
 //   warp 8     TMEM owner and MMA issuer (one elected lane): S = Q K^T into a
-//              double-buffered TMEM score tile, O += P V into TMEM.
+//              double-buffered TMEM score tile, O += P V into TMEM with P
+//              read from TMEM (the softmax writes P there, double-buffered).
+// K tiles (2 stages) are released as soon as S = Q K^T has read them, V tiles
+// (4 stages) once O += P V has, so the converters run up to four tiles ahead
+// of the P V products.
 // Both MMAs run in f16 with fp32 accumulation: every E4M3 value is exact in
 // f16, bf16 inputs are exact while inside f16's range (|x| <= 65504; below
 // 2^-14 they keep an absolute precision of 2^-24), and P gets 11 significant
@@ -44,32 +50,32 @@ constexpr int BM = 128;      // rows per CTA tile
 constexpr int BN = 128;      // keys per tile
 constexpr int kThreads = 288;
 constexpr int kSoftmaxWarps = 4, kMmaWarp = 8;  // warps 4-7 convert K/V
-constexpr uint32_t kTmemCols = 512;  // S[2] x 128 + O 128 -> 384, rounded to 2^k
+// TMEM columns: S[2] (2 x 128 fp32), O (128 fp32), P[2] (2 x 64 columns of f16 pairs)
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr int kOpBytes = BM * D * 2;  // one 128x128 16-bit operand = 32 KiB
+constexpr int kKStages = 2, kVStages = 4;
 constexpr int kQOff = 0;
-constexpr int kKOff = kQOff + kOpBytes;       // 2 stages
-constexpr int kVOff = kKOff + 2 * kOpBytes;   // 2 stages (V^T)
-constexpr int kPOff = kVOff + 2 * kOpBytes;
-constexpr int kStgOff = kPOff + kOpBytes;     // widened V, [key][d], 256-B rows
-constexpr int kBarOff = kStgOff + kOpBytes;
+constexpr int kKOff = kQOff + kOpBytes;              // K stages
+constexpr int kVOff = kKOff + kKStages * kOpBytes;   // V stages
+constexpr int kBarOff = kVOff + kVStages * kOpBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 
-// K-major operand with 128-byte swizzle: rows of 64 16-bit elements (128 B)
-// in two 16 KiB halves along K; chunk = 8 elements along K (0..15).
+// 128x128 16-bit operand with the 128-byte swizzle: 128-byte rows of 64
+// elements in two 16 KiB halves; chunk = 8 consecutive elements of a row
+// (0..15).  Read K-major (Q, K, P rows along K) or MN-major (V: rows are keys,
+// the 64-dim halves are the MN atoms, 8-row groups the K atoms).
 __device__ __forceinline__ uint32_t op_off(int row, int chunk) {
   return (chunk >> 3) * 16384 + row * 128 + ((((chunk & 7) ^ (row & 7))) << 4);
 }
-// staging [key][d] with the 32-byte granule XOR-ed by (key & 7)
-__device__ __forceinline__ uint32_t stg_off(int key, int d) {
-  return key * 256 + ((((d >> 4) ^ (key & 7))) << 5) + ((d & 15) << 1);
-}
-
 // ------------------------------------------------------------- tcgen05 ops
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+// shared-memory matrix descriptor, 128-byte swizzle: K-major operands use only
+// the 8-row group stride (1 KiB); the MN-major V operand also needs the stride
+// between its two 64-element MN halves (16 KiB) as the leading-dimension offset
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo = 16) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
@@ -78,6 +84,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, 
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+// same with A (M x K, 16-bit pairs along K in consecutive columns) read from TMEM
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                          uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum)
       : "memory");
 }
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -156,7 +171,8 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 struct Bars {
-  uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, pv_done, done;
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2], done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -209,14 +225,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x;
 
   if (tid == 0) {
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&B->k_full[s], 128);
+      mbar_init(&B->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&B->v_full[s], 128);
+      mbar_init(&B->v_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&B->kv_full[s], 128);
-      mbar_init(&B->kv_empty[s], 1);
       mbar_init(&B->s_full[s], 1);
       mbar_init(&B->s_empty[s], 128);
+      mbar_init(&B->p_full[s], 128);
+      mbar_init(&B->pv_done[s], 1);
     }
-    mbar_init(&B->p_full, 128);
-    mbar_init(&B->pv_done, 1);
     mbar_init(&B->done, 1);
     B->abort_flag = 0;
     fence_mbar_init();
@@ -247,20 +269,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 256;
+  const uint32_t tS = tmem, tO = tmem + 256, tP = tmem + 384;
 
   if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // kind::f16: D f32, A and B f16, both K-major, N = 128, M = 128
+      // kind::f16: D f32, A and B f16, N = 128, M = 128; B K-major for
+      // S = Q K^T, MN-major (bit 16) for O += P V
       const uint32_t idesc =
           (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-      const uint32_t aQ = sbase + kQOff, aP = sbase + kPOff;
+      const uint32_t idesc_pv = idesc | (1u << 16);
+      const uint32_t aQ = sbase + kQOff;
       bool ok = true;
       for (int j = 0; j <= nkt && ok; ++j) {
-        if (j < nkt) {
+        if (j < nkt) {  // S(j) = Q K(j)^T
           const int s = j & 1;
-          ok = wait_or_abort(&B->kv_full[s], (j >> 1) & 1, B, p.dev_err);
+          ok = wait_or_abort(&B->k_full[s], (j >> 1) & 1, B, p.dev_err);
           if (ok && j >= 2) ok = wait_or_abort(&B->s_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
           if (!ok) break;
           tc_fence_after();
@@ -271,20 +295,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_mma(tS + s * BN, smem_desc(aQ + off), smem_desc(bK + off), idesc, kk > 0);
           }
           tc_commit(&B->s_full[s]);
+          tc_commit(&B->k_empty[s]);  // the K stage is free once S(j) is done
         }
-        if (j >= 1) {
-          const int jp = j - 1, s = jp & 1;
-          ok = wait_or_abort(&B->p_full, jp & 1, B, p.dev_err);
+        if (j >= 1) {  // O += P(j-1) V(j-1), P from TMEM
+          const int jp = j - 1, b = jp & 1, sv = jp % kVStages;
+          ok = wait_or_abort(&B->v_full[sv], (jp / kVStages) & 1, B, p.dev_err);
+          if (ok) ok = wait_or_abort(&B->p_full[b], (jp >> 1) & 1, B, p.dev_err);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t bV = sbase + kVOff + s * kOpBytes;
+          const uint32_t bV = sbase + kVOff + sv * kOpBytes;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc_mma(tO, smem_desc(aP + off), smem_desc(bV + off), idesc, (jp > 0 || kk > 0));
+          for (int kk = 0; kk < BN / 16; ++kk) {  // 16 keys = two 8-row groups per step
+            tc_mma_ts(tO, tP + b * (BN / 2) + kk * 8, smem_desc(bV + kk * 2048, 16384),
+                      idesc_pv, (jp > 0 || kk > 0));
           }
-          tc_commit(&B->pv_done);
-          tc_commit(&B->kv_empty[s]);
+          tc_commit(&B->pv_done[b]);
+          tc_commit(&B->v_empty[sv]);
         }
       }
       // everything issued above has completed before TMEM is released
@@ -296,27 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ct = tid - kSoftmaxWarps * 32;  // 0..127
     const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
     const int kv_es = FP8 ? 1 : 2;
-    // K- and V-tile writers shared by both paths
-    auto write_v_transposed = [&](uint8_t* vop, const uint8_t* stg) {
-      // V^T: thread ct builds rows 2dp and 2dp+1 of the transposed tile for one
-      // half of the keys, reading both dims of a key with one 32-bit load
-      const int dp = ct & 63, kh = ct >> 6;
-#pragma unroll 2
-      for (int kc = kh * 8; kc < kh * 8 + 8; ++kc) {
-        uint32_t wa[4], wb[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k0 = kc * 8 + 2 * e;
-          const uint32_t u0 = *reinterpret_cast<const uint32_t*>(stg + stg_off(k0, 2 * dp));
-          const uint32_t u1 = *reinterpret_cast<const uint32_t*>(stg + stg_off(k0 + 1, 2 * dp));
-          wa[e] = __byte_perm(u0, u1, 0x5410u);  // (key k0, key k0+1) of dim 2dp
-          wb[e] = __byte_perm(u0, u1, 0x7632u);  // same keys of dim 2dp+1
-        }
-        *reinterpret_cast<uint4*>(vop + op_off(2 * dp, kc)) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-        *reinterpret_cast<uint4*>(vop + op_off(2 * dp + 1, kc)) =
-            make_uint4(wb[0], wb[1], wb[2], wb[3]);
-      }
-    };
     // block ids of a tile's 8 blocks (-1 past the context); the next tile's
     // are loaded a tile ahead so the K/V loads never wait on the block table
     auto load_ids = [&](int j, int (&ids)[8]) {
@@ -329,10 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int id_cur[8], id_nxt[8];
     load_ids(0, id_cur);
     for (int j = 0; j < nkt; ++j) {
-      const int s = j & 1;
+      const int s = j & 1, sv = j % kVStages;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
-      uint8_t* vop = smem + kVOff + s * kOpBytes;
-      uint8_t* stg = smem + kStgOff;
+      uint8_t* vop = smem + kVOff + sv * kOpBytes;
       if (j + 1 < nkt) load_ids(j + 1, id_nxt);
       // Each pass covers 128 x 16-byte chunks of stored K and V rows: for fp8,
       // pass m is block m of the tile (thread ct: key ct/8, chunk ct%8); for
@@ -363,9 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (g0 == 0) {
-          const bool stop =
-              j >= 2 && !wait_or_abort(&B->kv_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
+        if (g0 == 0) {  // the K stage is free once S(j-2) is done, the V stage once
+                        // O += P V of tile j-4 is
+          bool stop = j >= kKStages &&
+                      !wait_or_abort(&B->k_empty[s], ((j - kKStages) / kKStages) & 1, B, p.dev_err);
+          stop = stop || (j >= kVStages &&
+                          !wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1, B,
+                                         p.dev_err));
           if (conv_bar_or(stop || aborted(B))) goto conv_done;  // all converters stop together
         }
 #pragma unroll
@@ -383,32 +391,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 4; ++e) {
               kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
               kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
-              vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
-              vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
+              vh[2 * e] = e4m3x2_to_f16x2_div256(vw[e], 0x4140u);      // codes 0, 1
+              vh[2 * e + 1] = e4m3x2_to_f16x2_div256(vw[e], 0x4342u);  // codes 2, 3
             }
             *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc)) =
                 make_uint4(kh[0], kh[1], kh[2], kh[3]);
             *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc + 1)) =
                 make_uint4(kh[4], kh[5], kh[6], kh[7]);
-            *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc)) =
+            *reinterpret_cast<uint4*>(vop + op_off(key_t, 2 * cc)) =
                 make_uint4(vh[0], vh[1], vh[2], vh[3]);
-            *reinterpret_cast<uint4*>(stg + stg_off(key_t, 16 * cc + 8)) =
+            *reinterpret_cast<uint4*>(vop + op_off(key_t, 2 * cc + 1)) =
                 make_uint4(vh[4], vh[5], vh[6], vh[7]);
           } else {
             *reinterpret_cast<uint4*>(kop + op_off(key_t, cc)) =
                 make_uint4(bf16x2_to_f16x2(kr[u].x), bf16x2_to_f16x2(kr[u].y),
                            bf16x2_to_f16x2(kr[u].z), bf16x2_to_f16x2(kr[u].w));
-            *reinterpret_cast<uint4*>(stg + stg_off(key_t, 8 * cc)) =
+            *reinterpret_cast<uint4*>(vop + op_off(key_t, cc)) =
                 make_uint4(bf16x2_to_f16x2(vr[u].x), bf16x2_to_f16x2(vr[u].y),
                            bf16x2_to_f16x2(vr[u].z), bf16x2_to_f16x2(vr[u].w));
           }
         }
       }
-      conv_bar();
-      write_v_transposed(vop, stg);
       fence_async_smem();
-      mbar_arrive(&B->kv_full[s]);
-      conv_bar();  // staging is reused by the next tile
+      mbar_arrive(&B->k_full[s]);
+      mbar_arrive(&B->v_full[sv]);
 #pragma unroll
       for (int m = 0; m < 8; ++m) id_cur[m] = id_nxt[m];
     }
@@ -507,12 +513,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&B->s_empty[s]);  // S buffer s may be overwritten by S(j+2)
       l += rs;
-      // P and O are free once the previous tile's O += P V has completed
-      if (j >= 1) {
-        ok = __all_sync(0xffffffffu, wait_or_abort(&B->pv_done, (j - 1) & 1, B, p.dev_err));
+      const int b = j & 1;
+      // P buffer b is free once O += P V of tile j-2 has completed
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu,
+                        wait_or_abort(&B->pv_done[b], ((j - 2) >> 1) & 1, B, p.dev_err));
+        if (!ok) break;
+      }
+      // O is rescaled (rarely) once O += P V of tile j-1 has completed
+      if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
+        ok = __all_sync(0xffffffffu, wait_or_abort(&B->pv_done[b ^ 1], ((j - 1) >> 1) & 1, B,
+                                                   p.dev_err));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+        {
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             float o[32];
@@ -525,17 +539,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
       }
-      uint8_t* prow = smem + kPOff;
-#pragma unroll
-      for (int kc = 0; kc < BN / 8; ++kc)
-        *reinterpret_cast<uint4*>(prow + op_off(r, kc)) =
-            make_uint4(pk[4 * kc], pk[4 * kc + 1], pk[4 * kc + 2], pk[4 * kc + 3]);
-      fence_async_smem();
+      tc_fence_after();
+      // P row -> TMEM: column c of buffer b holds the f16 pair (key 2c, 2c+1)
+      tmem_st32(tP + lane_base + b * (BN / 2), reinterpret_cast<const float*>(pk));
+      tmem_st32(tP + lane_base + b * (BN / 2) + 32, reinterpret_cast<const float*>(pk + 32));
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&B->p_full);
+      mbar_arrive(&B->p_full[b]);
     }
     // epilogue: O / l after the last O += P V
-    if (ok && __all_sync(0xffffffffu, wait_or_abort(&B->pv_done, (nkt - 1) & 1, B, p.dev_err))) {
+    if (ok && __all_sync(0xffffffffu, wait_or_abort(&B->pv_done[(nkt - 1) & 1],
+                                                    ((nkt - 1) >> 1) & 1, B, p.dev_err))) {
       tc_fence_after();
       const float inv = (l > 0.f) ? p.out_mul / l : 0.f;
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) +
