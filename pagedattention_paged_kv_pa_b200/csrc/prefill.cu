@@ -331,13 +331,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         ids[m] = (blk * 16 < ctx) ? __ldg(&bt[blk]) : -1;
       }
     };
-    int id_cur[8], id_nxt[8];
+    int id_cur[8], id_nxt[8];  // ids of tile j and of tile j+1
     load_ids(0, id_cur);
+    if (nkt > 1) load_ids(1, id_nxt);
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1, sv = j % kVStages;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + sv * kOpBytes;
-      if (j + 1 < nkt) load_ids(j + 1, id_nxt);
+      // bulk-prefetch tile j+1's K and V blocks into L2, so that the loads of
+      // the next tile hit L2 instead of HBM
+      if (j + 1 < nkt && ct < 16) {
+        const int blk = (j + 1) * 8 + (ct & 7);
+        const int phys = blk * 16 < ctx ? __ldg(&bt[blk]) : -1;
+        if (phys >= 0 && phys < p.num_blocks)
+          prefetch_l2_bulk(static_cast<const uint8_t*>(ct < 8 ? k_pool : v_pool) +
+                               ((size_t)phys * p.n_kv + kvh) * 16 * D * kv_es,
+                           16 * D * kv_es);
+      }
       // Each pass covers 128 x 16-byte chunks of stored K and V rows: for fp8,
       // pass m is block m of the tile (thread ct: key ct/8, chunk ct%8); for
       // bf16, pass m is half of block m/2 (key 8(m%2) + ct/16, chunk ct%16).
@@ -417,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&B->v_full[sv]);
 #pragma unroll
       for (int m = 0; m < 8; ++m) id_cur[m] = id_nxt[m];
+      if (j + 2 < nkt) load_ids(j + 2, id_nxt);  // a whole tile ahead of its first use
     }
   conv_done:;
   } else {
