@@ -224,7 +224,7 @@ def run_ours(args, rank, world, local):
     kvdt = B.dtype_code(inp.k_pool)
     algo_bytes = W.decode_algorithmic_bytes(ctx, spec.n_q_heads, spec.n_kv_heads, spec.head_dim,
                                             W.ELEM_BYTES[spec.q_dtype], W.ELEM_BYTES[spec.kv_dtype])
-    n_parts = -(-mb * 16 // 512)
+    n_parts = -(-mb * 16 // (2048 if spec.kv_dtype == W.FP8_E4M3 else 1024))
     launches_per_step = 2 + (1 if n_parts > 1 else 0)
 
     def step(ev_a=None, ev_b=None):

@@ -108,11 +108,14 @@ const char* pa_status_string(pa_status s);
  * permutation of the physical blocks (partitioning and reduction order depend
  * only on logical positions).
  *
- * The work is split along the context into fixed partitions: a partition
- * kernel writes per-partition (max, sum, unnormalised output) into the
- * workspace and a reduce kernel merges the partitions of sequences that have
- * more than one.  pa_decode queues both; pa_decode_partitions and
- * pa_decode_reduce queue them one at a time (same arguments, same result).
+ * The work is split along the context into fixed partitions of 1024 tokens
+ * (16-bit and fp32 caches) or 2048 tokens (fp8 caches): a partition kernel
+ * writes per-partition (max, sum, unnormalised output) into the workspace and
+ * a reduce kernel merges the partitions of sequences that have more than one.
+ * pa_decode queues both; pa_decode_partitions and pa_decode_reduce queue them
+ * one at a time (same arguments, same result).  pa_decode_workspace_size does
+ * not depend on the dtypes (it is sized for 1024-token partitions) and is 0
+ * when every sequence fits one partition; the workspace may then be NULL.
  */
 size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim,
                                 int max_blocks_per_seq);

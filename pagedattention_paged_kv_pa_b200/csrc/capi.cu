@@ -167,7 +167,7 @@ const char* pa_status_string(pa_status s) {
 size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim, int max_blocks_per_seq) {
   if (num_seqs < 0 || n_q_heads < 1 || head_dim < 1 || max_blocks_per_seq < 1) return 0;
   DecodeShape s{n_q_heads, 1, head_dim, num_seqs, max_blocks_per_seq, 1,
-                pa::decode_num_parts(max_blocks_per_seq)};
+                pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   if (s.n_parts <= 1) return 0;
   return ws_total_bytes(s);
 }
@@ -180,7 +180,7 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
                                float k_scale, float v_scale, void* workspace,
                                size_t workspace_bytes, int32_t* dev_err, void* stream) {
   DecodeShape s{n_q_heads, n_kv_heads, head_dim, num_seqs, max_blocks_per_seq, num_blocks,
-                pa::decode_num_parts(max_blocks_per_seq)};
+                pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   pa_status st = check_decode(s, block_size, q_dtype, kv_dtype);
   if (st != PA_OK) return st;
   if (num_seqs == 0) return PA_OK;
@@ -190,7 +190,9 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
     return PA_ERR_INVALID_ARG;
   if (!(scale == scale) || (kv_dtype == PA_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)))
     return PA_ERR_INVALID_ARG;
-  if (s.n_parts > 1) {
+  // partitions this cache type uses; the workspace stride is s.n_parts
+  const int n_grid = pa::decode_num_parts(max_blocks_per_seq, pa::decode_part_tokens(kv_dtype));
+  if (n_grid > 1) {
     if (!workspace || !aligned16(workspace) || workspace_bytes < ws_total_bytes(s))
       return PA_ERR_INVALID_ARG;
   }
@@ -216,6 +218,7 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
   p.max_blocks = max_blocks_per_seq;
   p.num_blocks = num_blocks;
   p.n_parts_max = s.n_parts;
+  p.n_parts_grid = n_grid;
   CUtensorMap tmk, tmv;
   if (pa::decode_uses_tma(q_dtype, kv_dtype)) {
     if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
@@ -235,8 +238,9 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
   if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype) || q_dtype == PA_FP8_E4M3)
     return PA_ERR_INVALID_ARG;
   DecodeShape s{n_q_heads, 1, head_dim, num_seqs, max_blocks_per_seq, 1,
-                pa::decode_num_parts(max_blocks_per_seq)};
-  if (num_seqs == 0 || s.n_parts <= 1) return PA_OK;
+                pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
+  const int part_tokens = pa::decode_part_tokens(kv_dtype);
+  if (num_seqs == 0 || pa::decode_num_parts(max_blocks_per_seq, part_tokens) <= 1) return PA_OK;
   if (!out || !context_lens || !workspace || !aligned16(out) || !aligned16(workspace) ||
       workspace_bytes < ws_total_bytes(s))
     return PA_ERR_INVALID_ARG;
@@ -251,6 +255,7 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
   r.num_seqs = num_seqs;
   r.max_blocks = max_blocks_per_seq;
   r.n_parts_max = s.n_parts;
+  r.part_tokens = part_tokens;
   return cuda_status(pa::launch_decode_reduce(r, head_dim, q_dtype,
                                               static_cast<cudaStream_t>(stream)));
 }

@@ -8,7 +8,8 @@
 // goal is to keep enough bytes in flight and to touch every byte once.
 //
 // Split-context scheme.  Grid = (context partition, kv head, sequence); a
-// partition is kPart = 512 consecutive logical tokens (32 blocks).  Each CTA:
+// partition is 1024 consecutive logical tokens (64 blocks) with 16-bit caches
+// and 2048 with fp8 caches.  Each CTA:
 //   * one producer warp streams the partition's 16-token K and V tiles with
 //     2-D TMA loads (no multicast) into an 8-stage shared-memory ring guarded
 //     by mbarriers -- the block table indirection becomes one TMA row
@@ -41,12 +42,14 @@ namespace {
 
 constexpr int kNW = 4;  // consumer warps
 constexpr int kThreads = (kNW + 1) * 32;
-constexpr int kPartBlocks = kPart / 16;
 constexpr int kStages = 8;
 constexpr int kMaxGroup = 8;
 
 template <int D, bool FP8>
 struct MmaLayout {
+  static constexpr int kPart = FP8 ? kPartFp8 : kPart16;  // tokens per partition
+  static constexpr int kPartBlocks = kPart / 16;
+  static_assert(kPartBlocks <= kThreads, "one thread per block id");
   static constexpr int kTileBytes = 16 * D * (FP8 ? 1 : 2);  // one (block, head) tile
   static constexpr int kStageBytes = 2 * kTileBytes;          // K + V
   static constexpr int kIdsOff = kStages * kStageBytes;
@@ -151,6 +154,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   const int G = p.group;
   const int ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
                             threadIdx.x == 0 && part == 0 && kvh == 0);
+  constexpr int kPart = L::kPart;
   const int tok0 = part * kPart;
   if (tok0 >= ctx) {
     if (part == 0) {  // empty context: an all-zero output row
@@ -451,7 +455,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
 template <int D>
 __global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeParams p) {
   constexpr int VPL = D / 32;  // dims per lane
-  __shared__ int32_t ids[kPartBlocks];
+  constexpr int kPart = kPart16;
+  static_assert(kPart / 16 <= kNW * 32, "one thread per block id");
+  __shared__ int32_t ids[kPart / 16];
   __shared__ float mo[kNW * 8 * D];
   __shared__ float mm[kNW * 8], ml[kNW * 8], wgt[kNW * 8], Ls[8], Ms[8];
 
@@ -552,7 +558,7 @@ __global__ void __launch_bounds__(256) decode_reduce_kernel(const ReduceParams r
   const int seq = gw / r.n_q;
   int ctx = r.context_lens[seq];
   ctx = ctx < 0 ? 0 : min(ctx, r.max_blocks * 16);
-  const int np = (ctx + kPart - 1) / kPart;
+  const int np = (ctx + r.part_tokens - 1) / r.part_tokens;
   if (np <= 1) return;
   const float2* ml = r.ws_ml + (size_t)gw * r.n_parts_max;
   float M = -INFINITY;
@@ -594,22 +600,22 @@ cudaError_t launch_mma(const DecodeParams& p, const CUtensorMap* tmk, const CUte
   using L = MmaLayout<D, FP8>;
   static cudaError_t attr = set_smem(decode_mma_kernel<D, FP8, Q_BF16>, L::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  dim3 grid(p.n_parts_max, p.n_kv, p.num_seqs);
+  dim3 grid(p.n_parts_grid, p.n_kv, p.num_seqs);
   decode_mma_kernel<D, FP8, Q_BF16><<<grid, kThreads, L::kSmemBytes, st>>>(*tmk, *tmv, p);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_simt(const DecodeParams& p, cudaStream_t st) {
-  dim3 grid(p.n_parts_max, p.n_kv, p.num_seqs);
+  dim3 grid(p.n_parts_grid, p.n_kv, p.num_seqs);
   decode_simt_f32_kernel<D><<<grid, kNW * 32, 0, st>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int decode_num_parts(int max_blocks_per_seq) {
-  return (max_blocks_per_seq * 16 + kPart - 1) / kPart;
+int decode_num_parts(int max_blocks_per_seq, int part_tokens) {
+  return (int)(((int64_t)max_blocks_per_seq * 16 + part_tokens - 1) / part_tokens);
 }
 
 bool decode_uses_tma(pa_dtype q_dt, pa_dtype kv_dt) { return q_dt != PA_F32; }

@@ -1,8 +1,9 @@
 """GPU parity of pa_decode against the fp64 oracle on the same seeded inputs.
 
 Sizes are chosen so the oracle finishes in seconds while the GPU path still
-crosses many 16-token tiles, several 512-token partitions (so the reduce
-kernel runs) and a ragged last block.  Full-size workloads are checked on a
+crosses many 16-token tiles, several context partitions (1024 tokens with
+16-bit caches, 2048 with fp8 caches, so the reduce kernel runs) and a ragged
+last block.  Full-size workloads are checked on a
 sample of sequences in the launch configuration the benchmark times.
 """
 import numpy as np
@@ -40,7 +41,7 @@ def test_llama2_7b_fp16_reduced(B, cuda_device):
 
 def test_llama3_70b_gqa_bf16_reduced(B, cuda_device):
     spec = W.LLAMA3_70B_GQA_BF16.scaled(num_seqs=12)
-    ctx = np.array([16, 17, 511, 512, 513, 1000, 2048, 3001, 4096, 5555, 8191, 8192], np.int32)
+    ctx = np.array([16, 17, 1023, 1024, 1025, 1000, 2048, 3001, 4096, 5555, 8191, 8192], np.int32)
     _check(W.make_decode_inputs(spec, ctx=ctx), cuda_device, "llama3-70b bf16")
 
 
@@ -55,9 +56,10 @@ def test_fp8_cache_reduced(B, cuda_device):
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_dtype_group_headdim_grid(B, cuda_device, q_dt, kv_dt, d, G):
     n_kv = 2
-    ctx = np.array([0, 1, 2, 3, 5, 10, 15, 16, 17, 33, 500, 1100], np.int32)
+    # 1100 spans two 1024-token partitions, 2049 two 2048-token (fp8) ones
+    ctx = np.array([0, 1, 2, 3, 5, 10, 15, 16, 17, 33, 500, 1100, 2049], np.int32)
     spec = W.DecodeSpec("grid", len(ctx), n_kv * G, n_kv, d, q_dt, kv_dt, "fixed", (ctx,),
-                        max_ctx=1536, pool_factor=1.3, seed=77 + G + d)
+                        max_ctx=2304, pool_factor=1.3, seed=77 + G + d)
     inp = W.make_decode_inputs(spec, ctx=ctx)
     _check(inp, cuda_device, f"q={q_dt} kv={kv_dt} d={d} G={G}")
 
