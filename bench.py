@@ -519,20 +519,30 @@ def run_mixed(args, rank, world, local):
         dist.destroy_process_group()
 
 
+DECODE_SOURCES = ("decode.cu", "pa_internal.h", "pa_device.cuh")
+
+
+def decode_source_hash():
+    """First 16 hex digits of the SHA-256 of the decode kernel's sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        h.update(open(os.path.join(ROOT, "pagedattention_paged_kv_pa_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def traffic_from_profile(workload):
     """DRAM bytes per launch of the partition kernel from the committed ncu
     summary (profiles/decode_traffic.txt), if that summary was taken on the
-    current kernel source; None otherwise."""
-    import hashlib
+    current kernel sources; None otherwise."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.txt")
-    src = os.path.join(ROOT, "pagedattention_paged_kv_pa_b200", "csrc", "decode.cu")
     try:
         rec = {}
         for line in open(path):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 rec[k.strip()] = v.strip()
-        if rec.get("decode_cu_sha256_16") != hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]:
+        if rec.get("decode_src_sha256_16") != decode_source_hash():
             return None
         return int(rec[workload]) if workload in rec else None
     except Exception:

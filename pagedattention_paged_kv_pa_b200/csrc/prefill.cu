@@ -12,9 +12,9 @@
 // group).  Keys are processed in tiles of 128 (8 blocks of 16 from the block
 // table).  Warp roles (288 threads):
 //   warps 0-3  softmax: thread r owns row r = TMEM lane r; reads S from TMEM,
-//              masks, keeps an online max/sum, writes P (f16) to shared
-//              memory, rescales the TMEM output only when its max grew by more
-//              than 2^8, and writes the normalised output at the end;
+//              masks, keeps an online max/sum, writes P (f16) back to TMEM,
+//              rescales the TMEM output only when its max grew by more than
+//              2^8, and writes the normalised output at the end;
 //   warps 4-7  K/V converters: load a tile's K and V rows through the block
 //              table with coalesced 16-byte loads, widen fp8 codes exactly to
 //              f16 (K on the conversion pipe; V on the integer pipe as
@@ -33,7 +33,7 @@
 // 2^-14 they keep an absolute precision of 2^-24), and P gets 11 significant
 // bits instead of bf16's 8.
 // S(j+1) is issued before O += P(j) V(j), so the next tile's QK^T overlaps
-// this tile's softmax; K/V operands are double buffered.  All waits are
+// this tile's softmax.  All waits are
 // bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA drains its
 // tensor-core work and frees its TMEM before returning.
 #include <type_traits>
