@@ -15,6 +15,11 @@ replicas (weak scaling; decode needs no exchange between GPUs).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
+
+Other workloads: --workload mixed_step_fp8 (fp8-cache decode of 256 sequences
+next to a 2 x 512-query chunked prefill, on two streams) and --workload
+spec_verify_bf16 (the Llama-3-70B GQA cache with 5 new queries per sequence,
+pa_decode_multi, as when draft tokens are verified).
 """
 from __future__ import annotations
 
@@ -191,6 +196,50 @@ def oracle_sample(inp, budget_s: float, max_units=None):
         done_seqs += len(idx)
         done_tok += int(cl[idx].sum())
         s += len(idx)
+    return done_s, done_bytes, done_seqs, done_tok, threads
+
+
+def oracle_sample_multi(inp, qm, q_len: int, budget_s: float):
+    """Time the oracle's causal chunk (query i of a sequence with context c at
+    position c - q_len + i) on a bounded prefix of the sequences.
+    Returns (seconds, bytes, seqs, context tokens, threads)."""
+    import torch
+    import oracle as orc
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    spec = inp.spec
+    bt = inp.block_tables.cpu().numpy()
+    cl = inp.context_lens.cpu().numpy()
+    qc = qm.cpu()
+    threads = os.cpu_count() or 1
+    eb, qb = W.ELEM_BYTES[spec.kv_dtype], W.ELEM_BYTES[spec.q_dtype]
+    done_s, done_bytes, done_seqs, done_tok = 0.0, 0, 0, 0
+    s = 0
+    chunk = max(1, threads // max(1, spec.n_kv_heads) or 1)
+    while s < spec.num_seqs and done_s < budget_s:
+        idx = [i for i in range(s, min(s + chunk, spec.num_seqs)) if cl[i] > 0]
+        s = min(s + chunk, spec.num_seqs)
+        if not idx:
+            continue
+        need = sorted({int(b) for i in idx for b in bt[i, :-(-int(cl[i]) // 16)]})
+        remap = {b: j for j, b in enumerate(need)}
+        bt2 = np.full((len(idx), bt.shape[1]), -1, np.int32)
+        for r, i in enumerate(idx):
+            nb = -(-int(cl[i]) // 16)
+            bt2[r, :nb] = [remap[int(b)] for b in bt[i, :nb]]
+        sel = torch.tensor(need, dtype=torch.long, device=inp.k_pool.device)
+        k_sub, v_sub = inp.k_pool[sel].cpu(), inp.v_pool[sel].cpu()
+        m = [int(min(q_len, cl[i])) for i in idx]
+        qs = torch.cat([qc[i, q_len - k:] for i, k in zip(idx, m)])
+        qsl = np.concatenate([[0], np.cumsum(m)]).astype(np.int32)
+        t0 = time.perf_counter()
+        orc.paged_prefill(qs, k_sub, v_sub, bt2, qsl, cl[idx].astype(np.int32), inp.scale,
+                          spec.q_dtype, spec.kv_dtype, inp.k_scale, inp.v_scale,
+                          nthreads=threads)
+        done_s += time.perf_counter() - t0
+        done_bytes += (int(cl[idx].sum()) * 2 * spec.n_kv_heads * spec.head_dim * eb
+                       + len(idx) * q_len * spec.n_q_heads * spec.head_dim * 2 * qb)
+        done_seqs += len(idx)
+        done_tok += int(cl[idx].sum())
     return done_s, done_bytes, done_seqs, done_tok, threads
 
 
@@ -587,6 +636,150 @@ def run_reference(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def run_spec_verify(args, rank, world, local):
+    """Draft-token verification step on the Llama-3-70B GQA cache: the slot
+    write of each sequence's q_len new tokens, then pa_decode_multi (query i
+    of a sequence with context c attends to keys 0 .. c - q_len + i)."""
+    import torch
+    import oracle as orc
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_init(world, "nccl")
+    spec, q_len = W.SPEC_VERIFY_BF16, W.SPEC_VERIFY_Q_LEN
+    inp = W.make_decode_inputs(spec, device=dev)
+    qm = W.make_multi_queries(inp, q_len, seed=spec.seed + 1)
+    ctx = inp.context_lens.cpu().numpy()
+    n = spec.num_seqs
+    # the step's q_len new tokens of every sequence: positions c - q_len .. c - 1
+    pos = ctx[:, None] - q_len + np.arange(q_len)[None, :]
+    seq_ids = np.repeat(np.arange(n), q_len)
+    key, val = W.make_new_kv(n * q_len, spec.n_kv_heads, spec.head_dim, spec.kv_dtype, dev,
+                             seed=spec.seed + 7)
+    slots_np = W.slots_from_positions(inp.block_tables.cpu().numpy(), seq_ids,
+                                      np.maximum(pos.reshape(-1), 0))
+    slots_np[pos.reshape(-1) < 0] = -1
+    slots = torch.from_numpy(slots_np).to(dev)
+    out = torch.empty_like(qm)
+    mb = inp.block_tables.shape[1]
+    ws = torch.empty(max(B.pa_decode_workspace_size(n, spec.n_q_heads * q_len, spec.head_dim,
+                                                    mb), 16), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    eb = W.ELEM_BYTES[spec.kv_dtype]
+    qo_bytes = n * q_len * spec.n_q_heads * spec.head_dim * 2 * W.ELEM_BYTES[spec.q_dtype]
+    algo_bytes = int(ctx.sum()) * 2 * spec.n_kv_heads * spec.head_dim * eb + qo_bytes
+
+    def step(ev_a=None, ev_b=None):
+        B.pa_reshape_and_cache(inp.k_pool, inp.v_pool, key, val, slots, dev_err=err)
+        if ev_a is not None:
+            ev_a.record()
+        B.pa_decode_multi(out, qm, inp.k_pool, inp.v_pool, inp.block_tables, inp.context_lens,
+                          inp.scale, workspace=ws, dev_err=err)
+        if ev_b is not None:
+            ev_b.record()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    time.sleep(0.3)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    t0.record()
+    for i in range(K):
+        step(*evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clocks = sampler.stop()
+    ms_max = reduce_over_ranks(t0.elapsed_time(t1), "max", world, dev)
+    value = reduce_over_ranks(algo_bytes * K, "sum", world, dev) / (ms_max / 1e3) / 1e9
+    kern_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+
+    # ---- end to end through the public API from pinned host buffers
+    host = [t.cpu().pin_memory() for t in (qm, key, val, slots, inp.block_tables,
+                                            inp.context_lens)]
+    devb = [torch.empty_like(t) for t in (qm, key, val, slots, inp.block_tables,
+                                          inp.context_lens)]
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        for dst, src in zip(devb, host):
+            dst.copy_(src, non_blocking=True)
+        q_d, key_d, val_d, slots_d, bt_d, cl_d = devb
+        B.pa_reshape_and_cache(inp.k_pool, inp.v_pool, key_d, val_d, slots_d, dev_err=err)
+        B.pa_decode_multi(out, q_d, inp.k_pool, inp.v_pool, bt_d, cl_d, inp.scale,
+                          workspace=ws, dev_err=err)
+        out_h.copy_(out, non_blocking=True)
+
+    K2 = max(3, min(K, 200))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K2):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e2e_ms = reduce_over_ranks(e0.elapsed_time(e1), "max", world, dev)
+    e2e_value = reduce_over_ranks(algo_bytes * K2, "sum", world, dev) / (e2e_ms / 1e3) / 1e9
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+
+    peak, peak_src = hbm_peak()
+    achieved = algo_bytes / (kern_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) values, seeded context lengths and block shuffle)",
+        "config": {"workload": describe(spec, ctx, inp.num_blocks)
+                   + f"; {q_len} queries per sequence (draft-token verification)",
+                   "global_batch": n * world, "q_len": q_len, "seq_len": int(ctx.max()),
+                   "tokens_per_step": int(ctx.sum()), "algorithmic_bytes_per_step": algo_bytes,
+                   "step": f"reshape_and_cache ({q_len} new tokens/seq) + pa_decode_multi",
+                   "l2": "inputs larger than L2 (KV pool > 1 GB vs 126 MB L2); no flush",
+                   "parallelism": f"replicas x{world}"},
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": K2,
+                "ms_per_step": round(e2e_ms / K2, 4)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": traffic_from_profile("spec_verify_bf16"),
+                     "kernel": "pa_decode_multi (partition kernel + merge kernel)",
+                     "kernel_avg_us": round(kern_ms * 1e3, 2),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, b, ns, nt, th = oracle_sample_multi(inp, qm, q_len, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(b / secs / 1e9, 4), "unit": "GB/s", "cores": th,
+                                "kind": "oracle",
+                                "sample": f"first {ns} of {n} sequences ({nt} context tokens, "
+                                          f"{q_len} queries each) of the same workload, "
+                                          f"{secs:.1f} s, fp64 C oracle (causal chunk)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -602,6 +795,8 @@ def main(argv=None):
         run_reference(args, rank, world, local)
     elif args.workload == "mixed_step_fp8":
         run_mixed(args, rank, world, local)
+    elif args.workload == "spec_verify_bf16":
+        run_spec_verify(args, rank, world, local)
     else:
         run_ours(args, rank, world, local)
 

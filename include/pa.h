@@ -143,6 +143,40 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
                            const void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pa_decode_multi -- decode with q_len new queries per sequence, as when the
+ * target model verifies K draft tokens in one forward pass ([P1] §五
+ * "Speculative Decoding": the large model evaluates all K candidates in a
+ * single pass; [P3] "推測解碼": the k guessed tokens are checked in parallel).
+ * The K/V of all q_len tokens must already be in the cache
+ * (pa_reshape_and_cache), so context_lens[s] counts them; query i of sequence
+ * s (0 <= i < q_len) sits at position context_lens[s] - q_len + i and attends
+ * causally to keys 0 .. context_lens[s] - q_len + i:
+ *     out[s][i][h] = softmax(scale * q[s][i][h] . K_s[0..c_i]^T) . V_s[0..c_i]
+ * A query whose position is negative (context_lens[s] < q_len - i) has no
+ * keys and gets an all-zero row.  This is the causal chunk of
+ * pa_prefill_paged with history context_lens[s] - q_len, computed the way
+ * decode is: each K/V tile is read once for all of a sequence's queries of a
+ * kv head (up to 8 (query, head) pairs per tile pass), HBM-bound.
+ *
+ *   out, q       device [num_seqs][q_len][n_q_heads][head_dim], dtype q_dtype
+ *   q_len        1 .. 8 (1 gives pa_decode's result)
+ *   workspace    >= pa_decode_workspace_size(num_seqs, n_q_heads * q_len,
+ *                head_dim, max_blocks_per_seq) bytes, 16-byte aligned (may be
+ *                NULL when that size is 0)
+ *   other arguments as pa_decode.
+ *
+ * Supported as pa_decode except q_dtype PA_F32 (PA_ERR_UNSUPPORTED);
+ * q_len outside 1..8 is PA_ERR_INVALID_ARG.  Errors as pa_decode.
+ */
+pa_status pa_decode_multi(void* out, const void* q, const void* k_pool, const void* v_pool,
+                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                          int block_size, int n_q_heads, int n_kv_heads, int head_dim,
+                          int num_seqs, int q_len, int max_blocks_per_seq, int num_blocks,
+                          pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                          void* stream);
+
+/*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
  * memory and therefore have no workspace to pass: for example a plugin inside
  * a host program that owns all device memory and forbids cudaMalloc after

@@ -29,6 +29,7 @@ EXPORTS = (
     "pa_alloc_fork", "pa_alloc_prepare_write", "pa_alloc_free_seq", "pa_alloc_block_table",
     "pa_alloc_free_list", "pa_alloc_num_tokens", "pa_alloc_refcount", "pa_alloc_num_free",
     "pa_alloc_num_seqs", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
+    "pa_decode_multi",
 )
 
 
@@ -53,6 +54,8 @@ def _load() -> ctypes.CDLL:
     L.pa_decode.argtypes = dec
     L.pa_decode_partitions.argtypes = dec
     L.pa_decode_reduce.argtypes = [P, P, I, I, I, I, I, I, F, P, Z, P]
+    L.pa_decode_multi.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, F, F, P, Z,
+                                  P, P]
     L.pa_decode_noalloc.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, F, F, P, P]
     L.pa_decode_noalloc.restype = I
     L.pa_decode_noalloc_scratch_bytes.restype = Z
@@ -151,6 +154,30 @@ def _decode_args(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_sc
             float(scale), bs, n_q, n_kv, d, num_seqs, block_tables.shape[1], num_blocks,
             dtype_code(q), dtype_code(k_pool), float(k_scale), float(v_scale), _p(workspace),
             ws_bytes, _p(dev_err), _stream(stream, q.device))
+
+
+def pa_decode_multi(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale=1.0,
+                    v_scale=1.0, workspace=None, dev_err=None, stream=None):
+    """Multi-query decode: q / out are [num_seqs, q_len, n_q, d]; query i of a
+    sequence with context c attends to keys 0 .. c - q_len + i."""
+    _contig(out, q, k_pool, v_pool, block_tables, context_lens)
+    num_seqs, q_len, n_q, d = q.shape
+    num_blocks, n_kv, bs, d2 = k_pool.shape
+    if d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(out.shape) != tuple(q.shape):
+        raise PAError(PA_ERR_INVALID_ARG, "pa_decode_multi shapes")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise PAError(PA_ERR_INVALID_ARG, "block_tables / context_lens must be int32")
+    mb = block_tables.shape[1]
+    if workspace is None:
+        n = pa_decode_workspace_size(num_seqs, n_q * q_len, d, mb)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.pa_decode_multi(_p(out), _p(q), _p(k_pool), _p(v_pool), _p(block_tables),
+                               _p(context_lens), float(scale), bs, n_q, n_kv, d, num_seqs, q_len,
+                               mb, num_blocks, dtype_code(q), dtype_code(k_pool), float(k_scale),
+                               float(v_scale), _p(workspace), ws_bytes, _p(dev_err),
+                               _stream(stream, q.device)), "pa_decode_multi")
+    return out
 
 
 def pa_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale=1.0,

@@ -172,10 +172,10 @@ size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim, int m
   return ws_total_bytes(s);
 }
 
-pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, const void* v_pool,
+static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool, const void* v_pool,
                                const int32_t* block_tables, const int32_t* context_lens,
                                float scale, int block_size, int n_q_heads, int n_kv_heads,
-                               int head_dim, int num_seqs, int max_blocks_per_seq,
+                               int head_dim, int num_seqs, int q_len, int max_blocks_per_seq,
                                int num_blocks, pa_dtype q_dtype, pa_dtype kv_dtype,
                                float k_scale, float v_scale, void* workspace,
                                size_t workspace_bytes, int32_t* dev_err, void* stream) {
@@ -183,6 +183,12 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
                 pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   pa_status st = check_decode(s, block_size, q_dtype, kv_dtype);
   if (st != PA_OK) return st;
+  if (q_len < 1 || q_len > 8) return PA_ERR_INVALID_ARG;
+  if (q_len > 1 && q_dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+  const int n_cg = (n_q_heads / n_kv_heads * q_len + 7) / 8;  // column groups per kv head
+  if ((int64_t)n_kv_heads * n_cg > 65535) return PA_ERR_UNSUPPORTED;
+  DecodeShape ws = s;  // workspace rows: every (query, q head) of a sequence
+  ws.n_q = n_q_heads * q_len;
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
     return PA_ERR_INVALID_ARG;
@@ -193,7 +199,7 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
   // partitions this cache type uses; the workspace stride is s.n_parts
   const int n_grid = pa::decode_num_parts(max_blocks_per_seq, pa::decode_part_tokens(kv_dtype));
   if (n_grid > 1) {
-    if (!workspace || !aligned16(workspace) || workspace_bytes < ws_total_bytes(s))
+    if (!workspace || !aligned16(workspace) || workspace_bytes < ws_total_bytes(ws))
       return PA_ERR_INVALID_ARG;
   }
   const bool fp8 = kv_dtype == PA_FP8_E4M3;
@@ -206,7 +212,7 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
   p.context_lens = context_lens;
   p.ws_o = static_cast<float*>(workspace);
   p.ws_ml = workspace ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
-                                                  ((ws_o_bytes(s) + 255) & ~size_t(255)))
+                                                  ((ws_o_bytes(ws) + 255) & ~size_t(255)))
                       : nullptr;
   p.dev_err = dev_err;
   p.scale_log2 = scale * kLog2e * (fp8 ? k_scale : 1.f);
@@ -219,6 +225,8 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
   p.num_blocks = num_blocks;
   p.n_parts_max = s.n_parts;
   p.n_parts_grid = n_grid;
+  p.q_len = q_len;
+  p.n_cg = n_cg;
   CUtensorMap tmk, tmv;
   if (pa::decode_uses_tma(q_dtype, kv_dtype)) {
     if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
@@ -229,15 +237,28 @@ pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, con
                                                   static_cast<cudaStream_t>(stream)));
 }
 
-pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads, int head_dim,
+pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* block_tables, const int32_t* context_lens,
+                               float scale, int block_size, int n_q_heads, int n_kv_heads,
+                               int head_dim, int num_seqs, int max_blocks_per_seq,
+                               int num_blocks, pa_dtype q_dtype, pa_dtype kv_dtype,
+                               float k_scale, float v_scale, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  return decode_parts_impl(out, q, k_pool, v_pool, block_tables, context_lens, scale, block_size,
+                           n_q_heads, n_kv_heads, head_dim, num_seqs, 1, max_blocks_per_seq,
+                           num_blocks, q_dtype, kv_dtype, k_scale, v_scale, workspace,
+                           workspace_bytes, dev_err, stream);
+}
+
+static pa_status decode_reduce_impl(void* out, const int32_t* context_lens, int n_rows, int head_dim,
                            int num_seqs, int max_blocks_per_seq, pa_dtype q_dtype,
                            pa_dtype kv_dtype, float v_scale, const void* workspace,
                            size_t workspace_bytes, void* stream) {
   if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (num_seqs < 0 || n_q_heads < 1 || max_blocks_per_seq < 1) return PA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || n_rows < 1 || max_blocks_per_seq < 1) return PA_ERR_INVALID_ARG;
   if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype) || q_dtype == PA_FP8_E4M3)
     return PA_ERR_INVALID_ARG;
-  DecodeShape s{n_q_heads, 1, head_dim, num_seqs, max_blocks_per_seq, 1,
+  DecodeShape s{n_rows, 1, head_dim, num_seqs, max_blocks_per_seq, 1,
                 pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   const int part_tokens = pa::decode_part_tokens(kv_dtype);
   if (num_seqs == 0 || pa::decode_num_parts(max_blocks_per_seq, part_tokens) <= 1) return PA_OK;
@@ -251,13 +272,21 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
   r.ws_ml = reinterpret_cast<const float2*>(static_cast<const char*>(workspace) +
                                             ((ws_o_bytes(s) + 255) & ~size_t(255)));
   r.out_mul = kv_dtype == PA_FP8_E4M3 ? v_scale * kFp8VUnscale : 1.f;
-  r.n_q = n_q_heads;
+  r.n_q = n_rows;
   r.num_seqs = num_seqs;
   r.max_blocks = max_blocks_per_seq;
   r.n_parts_max = s.n_parts;
   r.part_tokens = part_tokens;
   return cuda_status(pa::launch_decode_reduce(r, head_dim, q_dtype,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads, int head_dim,
+                           int num_seqs, int max_blocks_per_seq, pa_dtype q_dtype,
+                           pa_dtype kv_dtype, float v_scale, const void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return decode_reduce_impl(out, context_lens, n_q_heads, head_dim, num_seqs, max_blocks_per_seq,
+                            q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
@@ -273,6 +302,23 @@ pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_
   if (st != PA_OK) return st;
   return pa_decode_reduce(out, context_lens, n_q_heads, head_dim, num_seqs, max_blocks_per_seq,
                           q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_multi(void* out, const void* q, const void* k_pool, const void* v_pool,
+                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                          int block_size, int n_q_heads, int n_kv_heads, int head_dim,
+                          int num_seqs, int q_len, int max_blocks_per_seq, int num_blocks,
+                          pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                          void* stream) {
+  pa_status st = decode_parts_impl(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                                   block_size, n_q_heads, n_kv_heads, head_dim, num_seqs, q_len,
+                                   max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                                   v_scale, workspace, workspace_bytes, dev_err, stream);
+  if (st != PA_OK) return st;
+  return decode_reduce_impl(out, context_lens, n_q_heads * q_len, head_dim, num_seqs,
+                            max_blocks_per_seq, q_dtype, kv_dtype, v_scale, workspace,
+                            workspace_bytes, stream);
 }
 
 pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,

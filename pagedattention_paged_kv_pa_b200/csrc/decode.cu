@@ -88,15 +88,28 @@ __device__ __forceinline__ int clamp_ctx(int ctx, int cap, int32_t* dev_err, boo
   return ctx < 0 ? 0 : ctx;
 }
 
+// Row of q / out (and of the workspace) that MMA column c of a CTA serves.  A
+// CTA's 8 columns are (query, head) pairs 8cg .. 8cg+7 of the sequence's
+// q_len x G pairs for its kv head, pair m being query m / G, head m % G of the
+// group; rows are laid out [seq][query][q head].  With one query per sequence
+// (decode) column c is simply head kvh*G + c.
+__device__ __forceinline__ size_t col_row(const DecodeParams& p, int seq, int kvh, int cg,
+                                          int c) {
+  const int m = 8 * cg + c, i = m / p.group;
+  return ((size_t)seq * p.q_len + i) * p.n_q + (size_t)kvh * p.group + (m - i * p.group);
+}
+
 // Merge the consumer warps' (m, l, O) states held in shared memory and write
-// the partition result.  mo: [kNW][8][D], mm/ml: [kNW][8] (log2-domain max and
-// running sum).  Called by every thread of the CTA.
+// the partition result of the CTA's ncols columns.  mo: [kNW][8][D], mm/ml:
+// [kNW][8] (log2-domain max and running sum).  Called by every thread of the
+// CTA.
 template <int D, typename OutT>
 __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml, float* wgt,
                                                 float* Ls, float* Ms, int nthreads,
                                                 const DecodeParams& p, int seq, int kvh,
-                                                int part, int n_parts_seq) {
-  const int G = p.group;
+                                                int cg, int ncols, int part,
+                                                int n_parts_seq) {
+  const int G = ncols;
   const int tid = threadIdx.x;
   if (tid < G) {
     float M = -INFINITY;
@@ -111,7 +124,6 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
     Ms[tid] = M;
   }
   __syncthreads();
-  const size_t head0 = (size_t)seq * p.n_q + (size_t)kvh * G;
   if (n_parts_seq == 1) {
     OutT* out = reinterpret_cast<OutT*>(p.out);
     for (int idx = tid; idx < G * D; idx += nthreads) {
@@ -120,7 +132,8 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
 #pragma unroll
       for (int w = 0; w < kNW; ++w) acc += wgt[w * 8 + h] * mo[(w * 8 + h) * D + dd];
       const float L = Ls[h];
-      out[(head0 + h) * D + dd] = from_f32<OutT>(L > 0.f ? acc / L * p.out_mul : 0.f);
+      out[col_row(p, seq, kvh, cg, h) * D + dd] =
+          from_f32<OutT>(L > 0.f ? acc / L * p.out_mul : 0.f);
     }
   } else {
     for (int idx = tid; idx < G * D; idx += nthreads) {
@@ -128,9 +141,10 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
       float acc = 0.f;
 #pragma unroll
       for (int w = 0; w < kNW; ++w) acc += wgt[w * 8 + h] * mo[(w * 8 + h) * D + dd];
-      p.ws_o[((head0 + h) * p.n_parts_max + part) * D + dd] = acc;
+      p.ws_o[(col_row(p, seq, kvh, cg, h) * p.n_parts_max + part) * D + dd] = acc;
     }
-    if (tid < G) p.ws_ml[(head0 + tid) * p.n_parts_max + part] = make_float2(Ms[tid], Ls[tid]);
+    if (tid < G)
+      p.ws_ml[col_row(p, seq, kvh, cg, tid) * p.n_parts_max + part] = make_float2(Ms[tid], Ls[tid]);
   }
 }
 
@@ -138,7 +152,10 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
 // tensor-core engine: 16-bit caches (MMA in the cache's type) and fp8 caches
 // (MMA in f16); Q_BF16 selects the query / output type.
 // ---------------------------------------------------------------------------
-template <int D, bool FP8, bool Q_BF16>
+// MQ: several queries per sequence (multi-query decode, e.g. verifying draft
+// tokens): query i of q_len sits at position ctx - q_len + i and sees keys
+// 0 .. ctx - q_len + i; blockIdx.y = kv head x column group.
+template <int D, bool FP8, bool Q_BF16, bool MQ>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
     const DecodeParams p) {
@@ -150,18 +167,20 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
-  const int part = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int part = blockIdx.x, seq = blockIdx.z;
+  const int kvh = MQ ? (int)blockIdx.y / p.n_cg : (int)blockIdx.y;
+  const int cg = MQ ? (int)blockIdx.y - kvh * p.n_cg : 0;
   const int G = p.group;
+  const int ncols = MQ ? min(8, G * p.q_len - 8 * cg) : G;  // columns in use
   const int ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
-                            threadIdx.x == 0 && part == 0 && kvh == 0);
+                            threadIdx.x == 0 && part == 0 && blockIdx.y == 0);
   constexpr int kPart = L::kPart;
   const int tok0 = part * kPart;
   if (tok0 >= ctx) {
-    if (part == 0) {  // empty context: an all-zero output row
+    if (part == 0) {  // empty context: all-zero output rows
       QT* out = reinterpret_cast<QT*>(p.out);
-      const size_t head0 = (size_t)seq * p.n_q + (size_t)kvh * G;
-      for (int idx = threadIdx.x; idx < G * D; idx += kThreads)
-        out[head0 * D + idx] = from_f32<QT>(0.f);
+      for (int idx = threadIdx.x; idx < ncols * D; idx += kThreads)
+        out[col_row(p, seq, kvh, cg, idx / D) * D + idx % D] = from_f32<QT>(0.f);
     }
     return;
   }
@@ -244,9 +263,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     // same pairing, which leaves the dot products unchanged.
     uint32_t qb[KS][2];
     {
-      const bool hv = g < G;
-      const QT* qrow = reinterpret_cast<const QT*>(p.q) +
-                       ((size_t)seq * p.n_q + (size_t)kvh * G + (hv ? g : 0)) * D;
+      const bool hv = g < ncols;
+      const QT* qrow = reinterpret_cast<const QT*>(p.q) + col_row(p, seq, kvh, cg, hv ? g : 0) * D;
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         if constexpr (FP8) {
@@ -263,6 +281,14 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     const float sl = p.scale_log2;
     const uint32_t sbase = smem_u32(smem);
     const int q4 = lane >> 3;
+    // multi-query causal limits: keys at positions >= lim are masked for the
+    // lane's two columns (2t, 2t+1); columns not in use keep the full context
+    int lim_a = ctx, lim_b = ctx;
+    const int lim_min = ctx - p.q_len + 1;  // the first query's limit
+    if constexpr (MQ) {
+      if (2 * t < ncols) lim_a = lim_min + (8 * cg + 2 * t) / G;
+      if (2 * t + 1 < ncols) lim_b = lim_min + (8 * cg + 2 * t + 1) / G;
+    }
 
     for (int j = warp; j < nblk; j += kNW) {
       const int s = j % kStages;
@@ -308,13 +334,27 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
           if (g >= valid) x0 = x1 = -INFINITY;
           if (g + 8 >= valid) x2 = x3 = -INFINITY;
         }
+        if constexpr (MQ) {
+          const int kb = tok0 + 16 * j;  // position of the block's first key
+          if (kb + 16 > lim_min) {
+            const int k0 = kb + g, k1 = k0 + 8;
+            if (k0 >= lim_a) x0 = -INFINITY;
+            if (k0 >= lim_b) x1 = -INFINITY;
+            if (k1 >= lim_a) x2 = -INFINITY;
+            if (k1 >= lim_b) x3 = -INFINITY;
+          }
+        }
         float b0m = fmaxf(x0, x2), b1m = fmaxf(x1, x3);
         b0m = warp_max_xor(b0m, 4);
         b1m = warp_max_xor(b1m, 4);
         const float n0 = fmaxf(m0, b0m), n1 = fmaxf(m1, b1m);
-        const float c0 = exp2f(m0 - n0), c1 = exp2f(m1 - n1);
-        const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1);
-        const float p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
+        // with several queries a column can have every key so far masked
+        // (max -inf); exponentiate against 0 then so that c = p = 0, not NaN
+        const float e0 = (MQ && n0 == -INFINITY) ? 0.f : n0;
+        const float e1 = (MQ && n1 == -INFINITY) ? 0.f : n1;
+        const float c0 = exp2f(m0 - e0), c1 = exp2f(m1 - e1);
+        const float p0 = exp2f(x0 - e0), p1 = exp2f(x1 - e1);
+        const float p2 = exp2f(x2 - e0), p3 = exp2f(x3 - e1);
         l0 = l0 * c0 + (p0 + p2);
         l1 = l1 * c1 + (p1 + p3);
         m0 = n0;
@@ -446,7 +486,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     }
   }
   __syncthreads();
-  merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, part, n_parts_seq);
+  merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, cg, ncols, part,
+                         n_parts_seq);
 }
 
 // ---------------------------------------------------------------------------
@@ -542,7 +583,8 @@ __global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeP
     }
   }
   __syncthreads();
-  merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, part, n_parts_seq);
+  merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, 0, G, part,
+                            n_parts_seq);
 }
 
 // ---------------------------------------------------------------------------
@@ -594,15 +636,22 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+template <int D, bool FP8, bool Q_BF16, bool MQ>
+cudaError_t launch_mma_(const DecodeParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                        cudaStream_t st) {
+  using L = MmaLayout<D, FP8>;
+  static cudaError_t attr = set_smem(decode_mma_kernel<D, FP8, Q_BF16, MQ>, L::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  dim3 grid(p.n_parts_grid, p.n_kv * (MQ ? p.n_cg : 1), p.num_seqs);
+  decode_mma_kernel<D, FP8, Q_BF16, MQ><<<grid, kThreads, L::kSmemBytes, st>>>(*tmk, *tmv, p);
+  return cudaGetLastError();
+}
+
 template <int D, bool FP8, bool Q_BF16>
 cudaError_t launch_mma(const DecodeParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
                        cudaStream_t st) {
-  using L = MmaLayout<D, FP8>;
-  static cudaError_t attr = set_smem(decode_mma_kernel<D, FP8, Q_BF16>, L::kSmemBytes);
-  if (attr != cudaSuccess) return attr;
-  dim3 grid(p.n_parts_grid, p.n_kv, p.num_seqs);
-  decode_mma_kernel<D, FP8, Q_BF16><<<grid, kThreads, L::kSmemBytes, st>>>(*tmk, *tmv, p);
-  return cudaGetLastError();
+  return p.q_len > 1 ? launch_mma_<D, FP8, Q_BF16, true>(p, tmk, tmv, st)
+                     : launch_mma_<D, FP8, Q_BF16, false>(p, tmk, tmv, st);
 }
 
 template <int D>

@@ -38,6 +38,8 @@ struct DecodeParams {
   int n_q, n_kv, group, num_seqs, max_blocks, num_blocks;
   int n_parts_max;   // workspace stride: partitions of max_blocks at kPart16
   int n_parts_grid;  // partitions of max_blocks at this cache type's length
+  int q_len;         // queries per sequence (1: decode; >1: multi-query decode)
+  int n_cg;          // groups of 8 (query, head) columns per kv head
 };
 
 struct ReduceParams {

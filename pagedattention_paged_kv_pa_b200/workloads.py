@@ -189,6 +189,15 @@ MIXED_DECODE_FP8 = DecodeSpec("mixed_step_fp8_decode", 256, 32, 8, 128, BF16, FP
 SPECS = {s.name: s for s in (TINY_FP32, LLAMA2_7B_FP16, LLAMA3_70B_GQA_BF16,
                              MIXED_DECODE_FP8)}
 
+# Draft-token verification ("LLM inference optimization", §五: the target model
+# checks K = 5 draft tokens in one forward pass): the Llama-3-70B GQA layer's
+# cache and contexts, with SPEC_VERIFY_Q_LEN new queries per sequence whose
+# K/V are the last SPEC_VERIFY_Q_LEN tokens of each context.
+SPEC_VERIFY_BF16 = DecodeSpec("spec_verify_bf16", 128, 64, 8, 128, BF16, BF16,
+                              "lognormal", (2048.0, 0.5, 16, 8192), max_ctx=8192,
+                              seed=1006)
+SPEC_VERIFY_Q_LEN = 5
+
 
 def context_lens_for(spec: DecodeSpec, rng) -> np.ndarray:
     if spec.ctx_kind == "fixed":
@@ -253,6 +262,15 @@ def make_decode_inputs(spec: DecodeSpec, device="cpu", ctx: Optional[np.ndarray]
     return DecodeInputs(spec, q, k_pool, v_pool,
                         torch.from_numpy(bt).to(device),
                         torch.from_numpy(ctx).to(device), scale, k_scale, v_scale)
+
+
+def make_multi_queries(inp: DecodeInputs, q_len: int, seed: int) -> torch.Tensor:
+    """Queries [num_seqs, q_len, n_q, d] for multi-query decode over inp's cache
+    (N(0,1) draws rounded to the query dtype)."""
+    spec = inp.spec
+    gen = _torch_gen(inp.k_pool.device, seed)
+    return randn_as((spec.num_seqs, q_len, spec.n_q_heads, spec.head_dim), spec.q_dtype,
+                    inp.k_pool.device, gen)
 
 
 # ----------------------------------------------------------------------------

@@ -86,6 +86,31 @@ def test_decode_argument_errors_are_synchronous(B):
     assert B.pa_decode_workspace_size(4, 8, 128, 32) == 0          # a single partition
 
 
+def _multi(B, q_len, **kw):
+    a = dict(out=16, q=16, k=16, v=16, bt=16, cl=16, scale=0.1, bs=16, nq=8, nkv=2, d=128,
+             ns=4, mb=4, nb=10, qdt=B.PA_BF16, kvdt=B.PA_BF16, ks=1.0, vs=1.0, ws=None,
+             wsb=0, err=None, st=None)
+    a.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return B.lib.pa_decode_multi(v(a["out"]), v(a["q"]), v(a["k"]), v(a["v"]), v(a["bt"]),
+                                 v(a["cl"]), a["scale"], a["bs"], a["nq"], a["nkv"], a["d"],
+                                 a["ns"], q_len, a["mb"], a["nb"], a["qdt"], a["kvdt"], a["ks"],
+                                 a["vs"], v(a["ws"]), a["wsb"], v(a["err"]), v(a["st"]))
+
+
+def test_multi_query_decode_argument_errors_are_synchronous(B):
+    assert _multi(B, 0) == B.PA_ERR_INVALID_ARG
+    assert _multi(B, 9) == B.PA_ERR_INVALID_ARG
+    assert _multi(B, 2, qdt=B.PA_F32, kvdt=B.PA_F32) == B.PA_ERR_UNSUPPORTED
+    assert _multi(B, 2, bs=32) == B.PA_ERR_UNSUPPORTED
+    assert _multi(B, 2, q=None) == B.PA_ERR_INVALID_ARG
+    assert _multi(B, 2, ns=0) == B.PA_OK
+    # the workspace holds every (query, q head) row of a sequence
+    ws = B.pa_decode_workspace_size(4, 8 * 3, 128, 512)
+    assert ws > 2 * B.pa_decode_workspace_size(4, 8, 128, 512)
+    assert _multi(B, 3, mb=512, ws=16, wsb=ws - 1) == B.PA_ERR_INVALID_ARG
+
+
 def test_cache_op_argument_errors_are_synchronous(B):
     v = ctypes.c_void_p
     L = B.lib
