@@ -55,7 +55,7 @@ struct MmaLayout {
   static constexpr int kIdsOff = kStages * kStageBytes;
   static constexpr int kBarOff = kIdsOff + kPartBlocks * 4;
   static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 1024;  // + align slack
-  static constexpr int kMergeFloats = kNW * kMaxGroup * D + 4 * kNW * kMaxGroup + 2 * kMaxGroup;
+  static constexpr int kMergeFloats = kNW * 8 * D + 3 * kNW * 8 + 2 * 32;
   static_assert(kMergeFloats * 4 <= kIdsOff, "merge scratch must fit in the ring");
   static_assert(kStageBytes % 1024 == 0, "1024-B aligned tiles");
 };
@@ -100,61 +100,65 @@ __device__ __forceinline__ size_t col_row(const DecodeParams& p, int seq, int kv
 }
 
 // Merge the consumer warps' (m, l, O) states held in shared memory and write
-// the partition result of the CTA's ncols columns.  mo: [kNW][8][D], mm/ml:
-// [kNW][8] (log2-domain max and running sum).  Called by every thread of the
-// CTA.
+// the partition result.  The CTA's nvc columns are "virtual columns"
+// vc = 8 gi + c of its column groups gi (group cg0 + gi of the sequence's
+// (query, head) pairs); group gi's state is spread over the wpg warps
+// w = gi + cpc2 * ph.  Plain decode: one group (cg0 = 0, cpc2 = 1) over all
+// kNW warps, nvc = G.  mo: [kNW][8][D], mm/ml/wgt: [kNW][8] (log2-domain max,
+// running sum, merge weight), Ls/Ms: [32].  Called by every thread of the CTA.
 template <int D, typename OutT>
 __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml, float* wgt,
                                                 float* Ls, float* Ms, int nthreads,
                                                 const DecodeParams& p, int seq, int kvh,
-                                                int cg, int ncols, int part,
+                                                int cg0, int cpc2, int wpg, int nvc, int part,
                                                 int n_parts_seq) {
-  const int G = ncols;
   const int tid = threadIdx.x;
-  if (tid < G) {
+  if (tid < nvc) {
+    const int gi = tid >> 3, c = tid & 7;
     float M = -INFINITY;
-    for (int w = 0; w < kNW; ++w) M = fmaxf(M, mm[w * 8 + tid]);
+    for (int ph = 0; ph < wpg; ++ph) M = fmaxf(M, mm[(gi + cpc2 * ph) * 8 + c]);
     float L = 0.f;
-    for (int w = 0; w < kNW; ++w) {
-      const float wv = (M == -INFINITY) ? 0.f : exp2f(mm[w * 8 + tid] - M);
-      wgt[w * 8 + tid] = wv;
-      L += wv * ml[w * 8 + tid];
+    for (int ph = 0; ph < wpg; ++ph) {
+      const int w = gi + cpc2 * ph;
+      const float wv = (M == -INFINITY) ? 0.f : exp2f(mm[w * 8 + c] - M);
+      wgt[w * 8 + c] = wv;
+      L += wv * ml[w * 8 + c];
     }
     Ls[tid] = L;
     Ms[tid] = M;
   }
   __syncthreads();
-  if (n_parts_seq == 1) {
-    OutT* out = reinterpret_cast<OutT*>(p.out);
-    for (int idx = tid; idx < G * D; idx += nthreads) {
-      const int h = idx / D, dd = idx % D;
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) acc += wgt[w * 8 + h] * mo[(w * 8 + h) * D + dd];
-      const float L = Ls[h];
-      out[col_row(p, seq, kvh, cg, h) * D + dd] =
+  for (int idx = tid; idx < nvc * D; idx += nthreads) {
+    const int vc = idx / D, dd = idx % D;
+    const int gi = vc >> 3, c = vc & 7;
+    float acc = 0.f;
+    for (int ph = 0; ph < wpg; ++ph) {
+      const int w = gi + cpc2 * ph;
+      acc += wgt[w * 8 + c] * mo[(w * 8 + c) * D + dd];
+    }
+    const size_t row = col_row(p, seq, kvh, cg0 + gi, c);
+    if (n_parts_seq == 1) {
+      const float L = Ls[vc];
+      reinterpret_cast<OutT*>(p.out)[row * D + dd] =
           from_f32<OutT>(L > 0.f ? acc / L * p.out_mul : 0.f);
+    } else {
+      p.ws_o[(row * p.n_parts_max + part) * D + dd] = acc;
     }
-  } else {
-    for (int idx = tid; idx < G * D; idx += nthreads) {
-      const int h = idx / D, dd = idx % D;
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) acc += wgt[w * 8 + h] * mo[(w * 8 + h) * D + dd];
-      p.ws_o[(col_row(p, seq, kvh, cg, h) * p.n_parts_max + part) * D + dd] = acc;
-    }
-    if (tid < G)
-      p.ws_ml[col_row(p, seq, kvh, cg, tid) * p.n_parts_max + part] = make_float2(Ms[tid], Ls[tid]);
   }
+  if (n_parts_seq > 1 && tid < nvc)
+    p.ws_ml[col_row(p, seq, kvh, cg0 + (tid >> 3), tid & 7) * p.n_parts_max + part] =
+        make_float2(Ms[tid], Ls[tid]);
 }
-
 // ---------------------------------------------------------------------------
 // tensor-core engine: 16-bit caches (MMA in the cache's type) and fp8 caches
 // (MMA in f16); Q_BF16 selects the query / output type.
 // ---------------------------------------------------------------------------
 // MQ: several queries per sequence (multi-query decode, e.g. verifying draft
 // tokens): query i of q_len sits at position ctx - q_len + i and sees keys
-// 0 .. ctx - q_len + i; blockIdx.y = kv head x column group.
+// 0 .. ctx - q_len + i.  A CTA takes up to 4 column groups of its kv head
+// (blockIdx.y = kv head x group quad); with cpc groups (cpc2 = cpc rounded up
+// to 1, 2 or 4) consumer warp w takes group w % cpc2 and every (4 / cpc2)-th
+// block, so one K/V stage serves all of the CTA's groups.
 template <int D, bool FP8, bool Q_BF16, bool MQ>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -168,10 +172,18 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   const int part = blockIdx.x, seq = blockIdx.z;
-  const int kvh = MQ ? (int)blockIdx.y / p.n_cg : (int)blockIdx.y;
-  const int cg = MQ ? (int)blockIdx.y - kvh * p.n_cg : 0;
   const int G = p.group;
-  const int ncols = MQ ? min(8, G * p.q_len - 8 * cg) : G;  // columns in use
+  int kvh = blockIdx.y, cg0 = 0, cpc = 1, cpc2 = 1;
+  if constexpr (MQ) {
+    const int nquad = (p.n_cg + 3) >> 2;
+    kvh = (int)blockIdx.y / nquad;
+    cg0 = 4 * ((int)blockIdx.y - kvh * nquad);
+    cpc = min(4, p.n_cg - cg0);
+    cpc2 = cpc == 1 ? 1 : (cpc == 2 ? 2 : 4);
+  }
+  const int wpg = kNW / cpc2;  // warps per column group
+  // virtual columns in use: 8 per full group, the last group's remainder
+  const int nvc = MQ ? min(8 * cpc, G * p.q_len - 8 * cg0) : G;
   const int ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
                             threadIdx.x == 0 && part == 0 && blockIdx.y == 0);
   constexpr int kPart = L::kPart;
@@ -179,8 +191,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   if (tok0 >= ctx) {
     if (part == 0) {  // empty context: all-zero output rows
       QT* out = reinterpret_cast<QT*>(p.out);
-      for (int idx = threadIdx.x; idx < ncols * D; idx += kThreads)
-        out[col_row(p, seq, kvh, cg, idx / D) * D + idx % D] = from_f32<QT>(0.f);
+      for (int idx = threadIdx.x; idx < nvc * D; idx += kThreads) {
+        const int vc = idx / D;
+        out[col_row(p, seq, kvh, cg0 + (vc >> 3), vc & 7) * D + idx % D] = from_f32<QT>(0.f);
+      }
     }
     return;
   }
@@ -204,7 +218,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], cpc);  // released by every group that reads the stage
     }
     fence_mbar_init();
   }
@@ -256,6 +270,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     }
   } else {
     // ------------------------------------------------------------ consumers
+    const int gi = warp % cpc2, ph = warp / cpc2;  // column group, block phase
+    const int cg = cg0 + gi;
+    const int ncols = MQ ? min(8, G * p.q_len - 8 * cg) : G;  // this warp's columns
+    const bool active = !MQ || gi < cpc;
     // Q as the B operand (k = head dim, n = query head of the group); heads
     // beyond the group size are zero.  The fp8 path pairs MMA k-index
     // (2t, 2t+1 | 2t+8, 2t+9) with dims (4t, 4t+1 | 4t+2, 4t+3) of each
@@ -290,7 +308,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
       if (2 * t + 1 < ncols) lim_b = lim_min + (8 * cg + 2 * t + 1) / G;
     }
 
-    for (int j = warp; j < nblk; j += kNW) {
+    for (int j = active ? ph : nblk; j < nblk; j += wpg) {
       const int s = j % kStages;
       if (!mbar_wait(&full[s], (j / kStages) & 1)) {
         flag_error(p.dev_err, PA_DEVERR_TIMEOUT);
@@ -465,7 +483,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   float* ml = mm + kNW * 8;
   float* wgt = ml + kNW * 8;
   float* Ls = wgt + kNW * 8;
-  float* Ms = Ls + 8;
+  float* Ms = Ls + 32;
   if (warp < kNW) {
     float* mw = mo + warp * 8 * D;
     // O^T row g / g+8 of m-tile i is dim 16i+g / 16i+g+8 (16-bit caches) or
@@ -486,8 +504,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     }
   }
   __syncthreads();
-  merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, cg, ncols, part,
-                         n_parts_seq);
+  merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, cg0, cpc2, wpg, nvc,
+                         part, n_parts_seq);
 }
 
 // ---------------------------------------------------------------------------
@@ -583,7 +601,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeP
     }
   }
   __syncthreads();
-  merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, 0, G, part,
+  merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, 0, 1, kNW, G, part,
                             n_parts_seq);
 }
 
@@ -642,7 +660,7 @@ cudaError_t launch_mma_(const DecodeParams& p, const CUtensorMap* tmk, const CUt
   using L = MmaLayout<D, FP8>;
   static cudaError_t attr = set_smem(decode_mma_kernel<D, FP8, Q_BF16, MQ>, L::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  dim3 grid(p.n_parts_grid, p.n_kv * (MQ ? p.n_cg : 1), p.num_seqs);
+  dim3 grid(p.n_parts_grid, p.n_kv * (MQ ? (p.n_cg + 3) / 4 : 1), p.num_seqs);
   decode_mma_kernel<D, FP8, Q_BF16, MQ><<<grid, kThreads, L::kSmemBytes, st>>>(*tmk, *tmv, p);
   return cudaGetLastError();
 }
