@@ -142,7 +142,8 @@ def test_free_returns_blocks_only_at_refcount_zero_fifo():
     assert m.free_seq("a") == OK
     assert m.num_free() == 3 and m.free_list() == [3, 4, 5]
     assert m.free_seq("b") == OK
-    assert m.free_list() == [3, 4, 5, 0, 1, 2]
+    # a finished request's blocks are released from its last block to its first
+    assert m.free_list() == [3, 4, 5, 2, 1, 0]
     assert m.free_seq("b") == INVALID_ARG
 
 
