@@ -304,6 +304,22 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_pairs,
  * queue, so the state after any call sequence is deterministic.  Every call is
  * all-or-nothing: PA_ERR_OOM or PA_ERR_INVALID_ARG leave the state unchanged.
  * Sequence ids are arbitrary int64 values.  Handles are not thread-safe.
+ *
+ * Prefix caching ([P2] "Prefix Caching：相同前綴只算一次"), off unless
+ * pa_alloc_set_prefix_caching switches it on: a block is in use (count > 0),
+ * free and empty, or free but holding cached content (count 0).  A full block
+ * whose token ids are known (pa_alloc_admit, pa_alloc_append_tokens) is
+ * registered under a 64-bit hash of its whole prefix, checked on a hit
+ * against its stored 16 tokens and its parent's hash.  pa_alloc_admit reuses
+ * the longest run of leading full blocks of a prompt held by a block in use
+ * or cached.  A new block is an empty one (FIFO) if any is left, else the
+ * least recently released cached block, whose registration is dropped; a
+ * block in use is never taken.  When a request ends, its registered blocks
+ * whose count reaches 0 become cached (the back of the LRU list) and the
+ * others empty.  A block whose prefix is already registered by another block
+ * stays unregistered; a partial last block is never registered.  Callers
+ * write the K/V of a registered block's tokens before any attention reads
+ * them (slot writes precede attention within a step).
  */
 typedef struct pa_alloc pa_alloc;
 
@@ -328,20 +344,46 @@ pa_status pa_alloc_fork(pa_alloc* a, int64_t parent, int64_t child);
 pa_status pa_alloc_prepare_write(pa_alloc* a, int64_t seq, int64_t* cow_pairs_out,
                                  int* n_pairs_out);
 
-/* Drop `seq`; each of its blocks' counts goes down by 1 and a block whose
- * count reaches 0 joins the back of the free queue (in logical order). */
+/* Drop `seq`; each of its blocks' counts goes down by 1, last block first,
+ * and a block whose count reaches 0 joins the back of the free queue (or,
+ * with prefix caching, of the cached list if it is registered). */
 pa_status pa_alloc_free_seq(pa_alloc* a, int64_t seq);
 
 /* Copy the block table of `seq` (logical order) into out[cap]; *n_out gets
  * its length.  PA_ERR_INVALID_ARG if cap is too small or seq is unknown. */
 pa_status pa_alloc_block_table(const pa_alloc* a, int64_t seq, int32_t* out, int cap,
                                int* n_out);
-/* Copy the free queue (front first) into out[cap]. */
+/* Copy the free queue of empty blocks (front first) into out[cap]. */
 pa_status pa_alloc_free_list(const pa_alloc* a, int32_t* out, int cap, int* n_out);
 int pa_alloc_num_tokens(const pa_alloc* a, int64_t seq); /* -1 if unknown */
 int pa_alloc_refcount(const pa_alloc* a, int32_t block); /* -1 if out of range */
-int pa_alloc_num_free(const pa_alloc* a);
+int pa_alloc_num_free(const pa_alloc* a);   /* empty free blocks */
 int pa_alloc_num_seqs(const pa_alloc* a);
+
+/* Switch prefix caching on (on != 0) or off; PA_ERR_INVALID_ARG while any
+ * sequence exists. */
+pa_status pa_alloc_set_prefix_caching(pa_alloc* a, int on);
+
+/* Start sequence `seq` (a new id) with a prompt of n_tokens known token ids.
+ * With prefix caching on, the longest run of the prompt's leading full blocks
+ * whose prefixes are registered is reused (counts + 1, cached blocks back in
+ * use); *n_cached_out = 16 x that run: those tokens' K/V are already in the
+ * cache and need no prefill.  The rest get new blocks.  slots_out[n_tokens]
+ * receives every token's slot, reused ones included.  PA_ERR_OOM when the new
+ * blocks cannot all be had (state unchanged). */
+pa_status pa_alloc_admit(pa_alloc* a, int64_t seq, const int32_t* tokens, int n_tokens,
+                         int64_t* slots_out, int* n_cached_out);
+
+/* pa_alloc_append for tokens whose ids are known: as long as every token of
+ * `seq` has come with its id, blocks it fills are registered.  (Plain
+ * pa_alloc_append makes a sequence's ids unknown from then on.) */
+pa_status pa_alloc_append_tokens(pa_alloc* a, int64_t seq, const int32_t* tokens,
+                                 int n_tokens, int64_t* slots_out);
+
+/* Copy the cached blocks (count 0, content kept), least recently released
+ * first, into out[cap]. */
+pa_status pa_alloc_cached_list(const pa_alloc* a, int32_t* out, int cap, int* n_out);
+int pa_alloc_num_cached(const pa_alloc* a);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,8 @@ EXPORTS = (
     "pa_alloc_fork", "pa_alloc_prepare_write", "pa_alloc_free_seq", "pa_alloc_block_table",
     "pa_alloc_free_list", "pa_alloc_num_tokens", "pa_alloc_refcount", "pa_alloc_num_free",
     "pa_alloc_num_seqs", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
-    "pa_decode_multi",
+    "pa_decode_multi", "pa_alloc_set_prefix_caching", "pa_alloc_admit",
+    "pa_alloc_append_tokens", "pa_alloc_cached_list", "pa_alloc_num_cached",
 )
 
 
@@ -82,8 +83,13 @@ def _load() -> ctypes.CDLL:
     L.pa_alloc_refcount.argtypes = [P, ctypes.c_int32]
     L.pa_alloc_num_free.argtypes = [P]
     L.pa_alloc_num_seqs.argtypes = [P]
+    L.pa_alloc_set_prefix_caching.argtypes = [P, I]
+    L.pa_alloc_admit.argtypes = [P, I64, P, I, P, P]
+    L.pa_alloc_append_tokens.argtypes = [P, I64, P, I, P]
+    L.pa_alloc_cached_list.argtypes = [P, P, I, P]
+    L.pa_alloc_num_cached.argtypes = [P]
     for fn in ("pa_alloc_num_tokens", "pa_alloc_refcount", "pa_alloc_num_free",
-               "pa_alloc_num_seqs"):
+               "pa_alloc_num_seqs", "pa_alloc_num_cached"):
         getattr(L, fn).restype = I
     return L
 
@@ -345,3 +351,36 @@ class BlockAllocator:
 
     def num_seqs(self) -> int:
         return lib.pa_alloc_num_seqs(self._h)
+
+    # -- prefix caching -------------------------------------------------------
+    def set_prefix_caching(self, on: bool) -> int:
+        return lib.pa_alloc_set_prefix_caching(self._h, 1 if on else 0)
+
+    def admit(self, seq: int, tokens):
+        """Returns (status, slots list, n_cached tokens)."""
+        n = len(tokens)
+        toks = (ctypes.c_int32 * max(n, 1))(*tokens)
+        buf = (ctypes.c_int64 * max(n, 1))()
+        nc = ctypes.c_int(0)
+        st = lib.pa_alloc_admit(self._h, seq, ctypes.cast(toks, ctypes.c_void_p), n,
+                                ctypes.cast(buf, ctypes.c_void_p), ctypes.byref(nc))
+        return st, (list(buf[:n]) if st == PA_OK else []), (nc.value if st == PA_OK else 0)
+
+    def append_tokens(self, seq: int, tokens):
+        """Returns (status, slots list)."""
+        n = len(tokens)
+        toks = (ctypes.c_int32 * max(n, 1))(*tokens)
+        buf = (ctypes.c_int64 * max(n, 1))()
+        st = lib.pa_alloc_append_tokens(self._h, seq, ctypes.cast(toks, ctypes.c_void_p), n,
+                                        ctypes.cast(buf, ctypes.c_void_p))
+        return st, (list(buf[:n]) if st == PA_OK else [])
+
+    def cached_list(self):
+        buf = (ctypes.c_int32 * self.num_blocks)()
+        n = ctypes.c_int(0)
+        _check(lib.pa_alloc_cached_list(self._h, ctypes.cast(buf, ctypes.c_void_p),
+                                        self.num_blocks, ctypes.byref(n)), "pa_alloc_cached_list")
+        return list(buf[:n.value])
+
+    def num_cached(self) -> int:
+        return lib.pa_alloc_num_cached(self._h)

@@ -75,3 +75,60 @@ def test_random_call_sequences_match_model(B, seed):
         else:
             assert a.free_seq(s) == m.free_seq(s)
         _same_state(a, m, seqs, N)
+
+
+@pytest.mark.parametrize("seed", [11, 12, 13, 14])
+def test_prefix_caching_call_sequences_match_model(B, seed):
+    """Prefix caching on: admissions drawn from a few shared prompts, token
+    appends, plain appends, forks, copy-on-write and frees; statuses, slots,
+    reused-token counts, free queue and cached (LRU) list agree after every
+    call."""
+    rnd = random.Random(seed)
+    N = rnd.choice([12, 24, 40])
+    order = rnd.sample(range(N), N)
+    a = B.BlockAllocator(N, 16, order)
+    m = AllocModel(N, 16, order)
+    assert a.set_prefix_caching(True) == m.set_prefix_caching(True) == 0
+    prompts = [[rnd.randrange(1 << 30) for _ in range(rnd.choice([16, 32, 40, 70]))]
+               for _ in range(6)]
+    seqs = list(range(40))
+    hits = 0
+    for _ in range(2000):
+        op = rnd.random()
+        s = rnd.choice(seqs)
+        if op < 0.3:
+            toks = list(rnd.choice(prompts))[:rnd.choice([16, 20, 32, 48, 70])]
+            toks += [rnd.randrange(1 << 30) for _ in range(rnd.choice([0, 1, 9, 16]))]
+            ra, rm = a.admit(s, toks), m.admit(s, toks)
+            assert ra == rm
+            hits += ra[2] > 0
+        elif op < 0.5:
+            toks = [rnd.randrange(1 << 30) for _ in range(rnd.choice([1, 5, 16, 23]))]
+            assert a.append_tokens(s, toks) == m.append_tokens(s, toks)
+        elif op < 0.55:
+            n = rnd.choice([1, 16])
+            ra, rm = a.append(s, n), m.append(s, n)
+            assert ra == (rm[0], rm[1])
+        elif op < 0.65:
+            c = rnd.choice(seqs)
+            assert a.fork(s, c) == m.fork(s, c)
+        elif op < 0.75:
+            ra, rm = a.prepare_write(s), m.prepare_write(s)
+            assert ra[0] == rm[0] and ra[1] == rm[1]
+        else:
+            assert a.free_seq(s) == m.free_seq(s)
+        _same_state(a, m, seqs, N)
+        assert a.cached_list() == m.cached_list()
+        assert a.num_cached() == len(m.cached)
+    assert hits > 20  # the walk exercised prefix reuse
+
+
+def test_prefix_caching_switch_and_admit_errors(B):
+    a = B.BlockAllocator(4, 16)
+    a.append(1, 3)
+    assert a.set_prefix_caching(True) == B.PA_ERR_INVALID_ARG
+    a.free_seq(1)
+    assert a.set_prefix_caching(True) == 0
+    assert a.admit(5, list(range(20)))[0] == 0
+    assert a.admit(5, list(range(20)))[0] == B.PA_ERR_INVALID_ARG   # id in use
+    assert a.admit(6, list(range(100)))[0] == B.PA_ERR_OOM
