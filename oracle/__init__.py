@@ -43,6 +43,8 @@ def lib():
         L.orc_reshape_and_cache.restype = I
         L.orc_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I]
         L.orc_copy_blocks.restype = I
+        L.orc_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I]
+        L.orc_swap_blocks.restype = I
         L.orc_decode_array.argtypes = [I, P, P, I64]
         L.orc_encode_e4m3_array.argtypes = [P, P, I64]
         L.orc_encode_bf16_array.argtypes = [P, P, I64]
@@ -150,6 +152,18 @@ def copy_blocks(k_pool: np.ndarray, v_pool: np.ndarray, pairs, dtype: int) -> in
 # --------------------------------------------------------------------------
 # number formats
 # --------------------------------------------------------------------------
+
+def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k, src_v, pairs, dtype: int) -> int:
+    """Copies block src of the source pools to block dst of the destination
+    pools for every (src, dst) pair, in place on dst; returns the number of
+    pairs skipped for an out-of-range id."""
+    assert dst_k.flags.c_contiguous and dst_v.flags.c_contiguous
+    sk, sv = _np(src_k), _np(src_v)
+    pr = np.ascontiguousarray(_np(pairs), dtype=np.int64).reshape(-1, 2)
+    dn, n_kv, bs, d = dst_k.shape
+    return lib().orc_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(sk), _ptr(sv), _ptr(pr), len(pr),
+                                 n_kv, d, bs, sk.shape[0], dn, dtype)
+
 
 def decode_values(codes, dtype: int) -> np.ndarray:
     a = _np(codes)

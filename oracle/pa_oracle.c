@@ -493,6 +493,30 @@ int orc_copy_blocks(void* k_pool, void* v_pool, const int64_t* pairs, int n_pair
     return bad;
 }
 
+/* Swap: copy whole blocks between two pools -- a GPU pool and a host pool,
+ * in either direction -- when a preempted request's KV cache is moved out
+ * and back ("vLLM explained", the table in "KV cache 什麼時候可以被覆蓋": when
+ * memory runs short, preempt by recomputation or by swapping to the CPU).
+ * For each pair (src, dst), block dst of the destination pools becomes a
+ * byte copy of block src of the source pools.  Pairs with an id out of range
+ * are skipped and counted. */
+int orc_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                    const int64_t* pairs, int n_pairs, int n_kv, int d, int block_size,
+                    int src_num_blocks, int dst_num_blocks, int dtype) {
+    int bad = 0;
+    size_t bytes = (size_t)n_kv * block_size * d * elem_bytes(dtype);
+    for (int p = 0; p < n_pairs; p++) {
+        int64_t s = pairs[2 * p], t = pairs[2 * p + 1];
+        if (s < 0 || s >= src_num_blocks || t < 0 || t >= dst_num_blocks) {
+            bad++;
+            continue;
+        }
+        memcpy((uint8_t*)dst_k + t * bytes, (const uint8_t*)src_k + s * bytes, bytes);
+        memcpy((uint8_t*)dst_v + t * bytes, (const uint8_t*)src_v + s * bytes, bytes);
+    }
+    return bad;
+}
+
 /* ------------------------------------------------------------------------ */
 /* array forms of the format routines (for exhaustive tests)                */
 /* ------------------------------------------------------------------------ */

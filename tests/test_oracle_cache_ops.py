@@ -87,6 +87,35 @@ def test_copy_blocks_copies_bytes_and_nothing_else():
     assert orc.copy_blocks(kp, vp, np.array([[0, 16], [-1, 3]], np.int64), orc.FP8_E4M3) == 2
 
 
+def test_swap_blocks_moves_blocks_between_pools():
+    # a preempted request's blocks go from the GPU pool to the host pool and
+    # back ("vLLM explained", "KV cache 什麼時候可以被覆蓋": swap to the CPU)
+    rng = np.random.default_rng(4)
+    for dt, shape, np_dt in ((orc.BF16, (12, 4, B, 64), np.uint16),
+                             (orc.FP8_E4M3, (12, 8, B, 128), np.uint8),
+                             (orc.F32, (12, 2, B, 64), np.uint32)):
+        gk = rng.integers(0, np.iinfo(np_dt).max, size=shape, dtype=np_dt)
+        gv = rng.integers(0, np.iinfo(np_dt).max, size=shape, dtype=np_dt)
+        hk = np.zeros((7,) + shape[1:], np_dt)
+        hv = np.zeros_like(hk)
+        out_pairs = np.array([[3, 0], [11, 6], [0, 2]], np.int64)
+        assert orc.swap_blocks(hk, hv, gk, gv, out_pairs, dt) == 0
+        for s, t in out_pairs:
+            assert np.array_equal(hk[t], gk[s]) and np.array_equal(hv[t], gv[s])
+        untouched = [i for i in range(7) if i not in (0, 6, 2)]
+        assert not hk[untouched].any() and not hv[untouched].any()
+        # back into other GPU blocks: the round trip is exact
+        back = np.array([[0, 5], [6, 9], [2, 1]], np.int64)
+        g0k, g0v = gk.copy(), gv.copy()
+        assert orc.swap_blocks(gk, gv, hk, hv, back, dt) == 0
+        for (s, _), (_, t) in zip(out_pairs, back):
+            assert np.array_equal(gk[t], g0k[s]) and np.array_equal(gv[t], g0v[s])
+        others = [i for i in range(12) if i not in (5, 9, 1)]
+        assert np.array_equal(gk[others], g0k[others]) and np.array_equal(gv[others], g0v[others])
+        # ids are checked against each pool's own size
+        assert orc.swap_blocks(hk, hv, gk, gv, np.array([[11, 7], [12, 0], [0, -1]]), dt) == 3
+
+
 # ---------------------------------------------------------------------------
 # allocator model
 # ---------------------------------------------------------------------------
