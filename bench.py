@@ -20,7 +20,9 @@ Other workloads: --workload mixed_step_fp8 (fp8-cache decode of 256 sequences
 next to a 2 x 512-query chunked prefill, on two streams) and --workload
 spec_verify_bf16 (the Llama-3-70B GQA cache with 5 new queries per sequence,
 pa_decode_multi, as when draft tokens are verified); --workload alloc_host
-(the host block allocator with prefix caching under a serving trace; no GPU).
+(the host block allocator with prefix caching under a serving trace; no GPU);
+--workload swap_bf16 (pa_swap_blocks moving 256 MB of blocks device <-> pinned
+host per direction).
 """
 from __future__ import annotations
 
@@ -781,6 +783,115 @@ def run_spec_verify(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def run_swap(args, rank, world, local):
+    """Swap preemption's data path: 4,096 blocks of the Llama-3-70B GQA layer
+    (8 kv heads x 16 tokens x 128 dims, bf16, K and V: 256 MB) from the device
+    pool to a pinned host pool and 4,096 back, per step, with pa_swap_blocks
+    (one kernel per direction; the pair lists live in pinned host memory).
+    The roofline denominator is a contiguous 256 MB pinned-host <-> device
+    copy measured in the same run (the host link's copy-engine rate)."""
+    import torch
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_init(world, "nccl")
+    n_kv, d, n_dev, n_host, n_move = 8, 128, 8192, 4096, 4096
+    shape = (n_dev, n_kv, 16, d)
+    kp = torch.randn(shape, dtype=torch.bfloat16, device=dev)
+    vp = torch.randn(shape, dtype=torch.bfloat16, device=dev)
+    hk = torch.empty((n_host,) + shape[1:], dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    rng = np.random.default_rng(1008)
+    out_pairs = torch.from_numpy(np.stack([rng.permutation(n_dev)[:n_move],
+                                           np.arange(n_move)], 1).astype(np.int64)).pin_memory()
+    in_pairs = torch.from_numpy(np.stack([np.arange(n_move), rng.permutation(n_dev)[:n_move]],
+                                         1).astype(np.int64)).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    block_bytes = n_kv * 16 * d * 2
+    moved = 2 * n_move * block_bytes  # K and V, one direction
+
+    def step(evs=None):
+        if evs:
+            evs[0].record()
+        B.pa_swap_blocks(hk, hv, kp, vp, out_pairs, dev_err=err)
+        if evs:
+            evs[1].record()
+        B.pa_swap_blocks(kp, vp, hk, hv, in_pairs, dev_err=err)
+        if evs:
+            evs[2].record()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+    # the host link's contiguous copy rate, each direction
+    flat_d = torch.empty(moved // 2, dtype=torch.bfloat16, device=dev)
+    flat_h = torch.empty(moved // 2, dtype=torch.bfloat16).pin_memory()
+    ref = {}
+    for name, fn in (("d2h", lambda: flat_h.copy_(flat_d, non_blocking=True)),
+                     ("h2d", lambda: flat_d.copy_(flat_h, non_blocking=True))):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(5):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ref[name] = moved / (a.elapsed_time(b) / 5 / 1e3) / 1e9
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K):
+        step(evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clocks = sampler.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+    ms = reduce_over_ranks(t0.elapsed_time(t1), "max", world, dev)
+    out_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    in_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    value = reduce_over_ranks(2 * moved * K, "sum", world, dev) / (ms / 1e3) / 1e9
+    out_gbs, in_gbs = moved / (out_ms / 1e3) / 1e9, moved / (in_ms / 1e3) / 1e9
+    line = {
+        "metric": "KV block swap GB/s (device <-> pinned host, both directions)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"swap out {n_move} and in {n_move} random blocks of a "
+                               f"{n_dev}-block device pool via a {n_host}-block pinned host "
+                               f"pool; block = {n_kv} kv heads x 16 tokens x {d} dims bf16, "
+                               f"K and V ({2 * block_bytes} B)",
+                   "bytes_per_direction": moved, "parallelism": f"replicas x{world}"},
+        "swap_out": {"us": round(out_ms * 1e3, 1), "gbs": round(out_gbs, 2),
+                     "contiguous_copy_gbs": round(ref["d2h"], 2),
+                     "frac": round(out_gbs / ref["d2h"], 4)},
+        "swap_in": {"us": round(in_ms * 1e3, 1), "gbs": round(in_gbs, 2),
+                    "contiguous_copy_gbs": round(ref["h2d"], 2),
+                    "frac": round(in_gbs / ref["h2d"], 4)},
+        "roofline": {"bound": "host_link", "achieved": round(min(out_gbs, in_gbs), 2),
+                     "peak": round(min(ref["d2h"], ref["h2d"]), 2), "unit": "GB/s",
+                     "frac": round(min(out_gbs / ref["d2h"], in_gbs / ref["h2d"]), 4),
+                     "traffic": None, "kernel": "copy_blocks_kernel (pa_swap_blocks)",
+                     "peak_source": "contiguous pinned-host <-> device copy, same run"},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def run_alloc_host(args):
     """Host allocator under a synthetic serving trace (no GPU): requests drawn
     from 8 shared system prompts (256-1024 tokens) plus 16-256 private tokens
@@ -851,6 +962,8 @@ def main(argv=None):
         run_spec_verify(args, rank, world, local)
     elif args.workload == "alloc_host":
         run_alloc_host(args)
+    elif args.workload == "swap_bf16":
+        run_swap(args, rank, world, local)
     else:
         run_ours(args, rank, world, local)
 

@@ -288,6 +288,34 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_pairs,
                          int n_kv_heads, int head_dim, int block_size, int num_blocks,
                          pa_dtype kv_dtype, int32_t* dev_err, void* stream);
 
+/*
+ * pa_swap_blocks -- move whole blocks between two pools, e.g. a preempted
+ * request's blocks from the GPU pool to a host pool and later back ([P2]
+ * "KV cache 什麼時候可以被覆蓋": when memory runs short a request is
+ * preempted by recomputation or by swapping its KV cache to the CPU).  For
+ * each pair (src, dst), block dst of (dst_k_pool, dst_v_pool) becomes a byte
+ * copy of block src of (src_k_pool, src_v_pool), every KV head, K and V.  One
+ * kernel moves all pairs; host blocks cross the host link as the kernel's own
+ * loads and stores.
+ *
+ *   pools        each either memory of the current device or pinned host
+ *                memory mapped into the device's address space (cudaHostAlloc
+ *                / cudaMallocHost, or cudaHostRegister with
+ *                cudaHostRegisterMapped), [num_blocks][n_kv][16][head_dim],
+ *                16-byte aligned; src and dst pools must not overlap
+ *   block_pairs  int64 [n_pairs][2] = (src, dst) in the same kinds of memory;
+ *                dst ids distinct.  Ids outside [0, src_num_blocks) /
+ *                [0, dst_num_blocks) are skipped and flagged with
+ *                PA_DEVERR_SLOT.
+ * Pointers to pageable host memory or to another GPU's memory are refused
+ * with PA_ERR_INVALID_ARG before any launch.
+ */
+pa_status pa_swap_blocks(void* dst_k_pool, void* dst_v_pool, const void* src_k_pool,
+                         const void* src_v_pool, const int64_t* block_pairs, int n_pairs,
+                         int n_kv_heads, int head_dim, int block_size, int src_num_blocks,
+                         int dst_num_blocks, pa_dtype kv_dtype, int32_t* dev_err,
+                         void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* Host block allocator (not on the hot path)                                 */
 /* ------------------------------------------------------------------------- */

@@ -31,6 +31,7 @@ EXPORTS = (
     "pa_alloc_num_seqs", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
     "pa_decode_multi", "pa_alloc_set_prefix_caching", "pa_alloc_admit",
     "pa_alloc_append_tokens", "pa_alloc_cached_list", "pa_alloc_num_cached",
+    "pa_swap_blocks",
 )
 
 
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
     L.pa_alloc_refcount.argtypes = [P, ctypes.c_int32]
     L.pa_alloc_num_free.argtypes = [P]
     L.pa_alloc_num_seqs.argtypes = [P]
+    L.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.pa_alloc_set_prefix_caching.argtypes = [P, I]
     L.pa_alloc_admit.argtypes = [P, I64, P, I, P, P]
     L.pa_alloc_append_tokens.argtypes = [P, I64, P, I, P]
@@ -279,6 +281,25 @@ def pa_copy_blocks(k_pool, v_pool, block_pairs, dev_err=None, stream=None):
     _check(lib.pa_copy_blocks(_p(k_pool), _p(v_pool), _p(block_pairs), n_pairs, n_kv, d, bs,
                               num_blocks, dtype_code(k_pool), _p(dev_err),
                               _stream(stream, k_pool.device)), "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_pairs, dev_err=None, stream=None):
+    """Block dst of (dst_k, dst_v) := block src of (src_k, src_v) for every
+    (src, dst) row of block_pairs.  Each pool (and block_pairs) is a tensor on
+    the current CUDA device or a pinned CPU tensor."""
+    _contig(dst_k, dst_v, src_k, src_v, block_pairs)
+    if block_pairs.dtype != torch.int64:
+        raise PAError(PA_ERR_INVALID_ARG, "block_pairs must be int64 [n][2]")
+    dn, n_kv, bs, d = dst_k.shape
+    sn = src_k.shape[0]
+    if tuple(src_k.shape[1:]) != (n_kv, bs, d) or dst_v.shape != dst_k.shape or \
+            src_v.shape != src_k.shape or dtype_code(src_k) != dtype_code(dst_k):
+        raise PAError(PA_ERR_INVALID_ARG, "pa_swap_blocks pool shapes")
+    dev = next((t.device for t in (dst_k, src_k, block_pairs) if t.is_cuda),
+               torch.device("cuda", torch.cuda.current_device()))
+    _check(lib.pa_swap_blocks(_p(dst_k), _p(dst_v), _p(src_k), _p(src_v), _p(block_pairs),
+                              block_pairs.numel() // 2, n_kv, d, bs, sn, dn, dtype_code(dst_k),
+                              _p(dev_err), _stream(stream, dev)), "pa_swap_blocks")
 
 
 # --------------------------------------------------------------------------

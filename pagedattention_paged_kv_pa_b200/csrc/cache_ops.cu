@@ -73,31 +73,36 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const ScatterPar
   }
 }
 
-// grid = (pair, K-or-V, 16 KiB piece of the block); 256 threads x 4 x 16 B.
+// grid = (pairs, K-or-V, 16 KiB piece of the block); 256 threads x 4 x 16 B,
+// the x dimension striding over the pairs.  Either pool may be pinned host
+// memory mapped into the device address space (swapping); its bytes then
+// cross the host link in 512-byte warp-wide requests.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(const CopyParams p) {
-  const int pair = blockIdx.x;
-  const int64_t s = p.pairs[2 * pair], d = p.pairs[2 * pair + 1];
-  if (s < 0 || s >= p.num_blocks || d < 0 || d >= p.num_blocks) {
-    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-      flag_error(p.dev_err, PA_DEVERR_SLOT);
-    return;
-  }
-  uint8_t* pool = reinterpret_cast<uint8_t*>(blockIdx.y ? p.v_pool : p.k_pool);
-  const uint4* src = reinterpret_cast<const uint4*>(pool + s * p.block_bytes);
-  uint4* dst = reinterpret_cast<uint4*>(pool + d * p.block_bytes);
+  const uint8_t* spool = reinterpret_cast<const uint8_t*>(blockIdx.y ? p.src_v : p.src_k);
+  uint8_t* dpool = reinterpret_cast<uint8_t*>(blockIdx.y ? p.dst_v : p.dst_k);
   const int64_t n16 = p.block_bytes / 16;
   const int64_t lo = (int64_t)blockIdx.z * 1024;
   const int64_t hi = lo + 1024 < n16 ? lo + 1024 : n16;
-  uint4 v[4];
+  for (int pair = blockIdx.x; pair < p.n_pairs; pair += gridDim.x) {
+    const int64_t s = p.pairs[2 * pair], d = p.pairs[2 * pair + 1];
+    if (s < 0 || s >= p.src_num_blocks || d < 0 || d >= p.dst_num_blocks) {
+      if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+        flag_error(p.dev_err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(spool + s * p.block_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(dpool + d * p.block_bytes);
+    uint4 v[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int64_t idx = lo + threadIdx.x + 256 * k;
-    if (idx < hi) v[k] = src[idx];
-  }
+    for (int k = 0; k < 4; ++k) {
+      const int64_t idx = lo + threadIdx.x + 256 * k;
+      if (idx < hi) v[k] = src[idx];
+    }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int64_t idx = lo + threadIdx.x + 256 * k;
-    if (idx < hi) dst[idx] = v[k];
+    for (int k = 0; k < 4; ++k) {
+      const int64_t idx = lo + threadIdx.x + 256 * k;
+      if (idx < hi) dst[idx] = v[k];
+    }
   }
 }
 
@@ -128,7 +133,7 @@ cudaError_t launch_reshape_and_cache(const ScatterParams& p, pa_dtype src_dt, pa
 cudaError_t launch_copy_blocks(const CopyParams& p, cudaStream_t st) {
   if (p.n_pairs == 0) return cudaSuccess;
   const int64_t n16 = p.block_bytes / 16;
-  dim3 grid(p.n_pairs, 2, (unsigned)((n16 + 1023) / 1024));
+  dim3 grid(p.n_pairs < 65535 ? p.n_pairs : 65535, 2, (unsigned)((n16 + 1023) / 1024));
   copy_blocks_kernel<<<grid, 256, 0, st>>>(p);
   return cudaGetLastError();
 }

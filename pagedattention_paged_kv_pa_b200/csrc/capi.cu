@@ -408,19 +408,70 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int64_t* block_pairs,
   if (block_size != 16) return PA_ERR_UNSUPPORTED;
   if (n_pairs < 0 || n_kv_heads < 1 || head_dim < 1 || num_blocks < 1 || !valid_dtype(kv_dtype))
     return PA_ERR_INVALID_ARG;
-  if (n_pairs > 65535) return PA_ERR_UNSUPPORTED;
   const int64_t bb = (int64_t)n_kv_heads * 16 * head_dim * elem_bytes(kv_dtype);
   if (bb % 16 != 0) return PA_ERR_UNSUPPORTED;
   if (n_pairs == 0) return PA_OK;
   if (!k_pool || !v_pool || !block_pairs || !aligned16(k_pool) || !aligned16(v_pool))
     return PA_ERR_INVALID_ARG;
   pa::CopyParams p;
-  p.k_pool = k_pool;
-  p.v_pool = v_pool;
+  p.dst_k = k_pool;
+  p.dst_v = v_pool;
+  p.src_k = k_pool;
+  p.src_v = v_pool;
   p.pairs = block_pairs;
   p.dev_err = dev_err;
   p.n_pairs = n_pairs;
-  p.num_blocks = num_blocks;
+  p.src_num_blocks = p.dst_num_blocks = num_blocks;
+  p.block_bytes = bb;
+  return cuda_status(pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream)));
+}
+
+// The address a kernel on the current device uses for `ptr`, which must be
+// memory of that device or pinned host memory mapped into its address space
+// (cudaHostAlloc / cudaMallocHost, or cudaHostRegister with
+// cudaHostRegisterMapped); NULL for anything else (pageable host memory,
+// another GPU's memory), which a kernel could not touch safely.
+static const void* device_view(const void* ptr) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();  // clear the error this query left, so a later launch check is clean
+    return nullptr;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (a.type == cudaMemoryTypeDevice) return a.device == dev ? ptr : nullptr;
+  if (a.type == cudaMemoryTypeHost || a.type == cudaMemoryTypeManaged) return a.devicePointer;
+  return nullptr;
+}
+
+pa_status pa_swap_blocks(void* dst_k_pool, void* dst_v_pool, const void* src_k_pool,
+                         const void* src_v_pool, const int64_t* block_pairs, int n_pairs,
+                         int n_kv_heads, int head_dim, int block_size, int src_num_blocks,
+                         int dst_num_blocks, pa_dtype kv_dtype, int32_t* dev_err,
+                         void* stream) {
+  if (block_size != 16) return PA_ERR_UNSUPPORTED;
+  if (n_pairs < 0 || n_kv_heads < 1 || head_dim < 1 || src_num_blocks < 1 ||
+      dst_num_blocks < 1 || !valid_dtype(kv_dtype))
+    return PA_ERR_INVALID_ARG;
+  const int64_t bb = (int64_t)n_kv_heads * 16 * head_dim * elem_bytes(kv_dtype);
+  if (bb % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (n_pairs == 0) return PA_OK;
+  if (!dst_k_pool || !dst_v_pool || !src_k_pool || !src_v_pool || !block_pairs)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(dst_k_pool) || !aligned16(dst_v_pool) || !aligned16(src_k_pool) ||
+      !aligned16(src_v_pool) || (reinterpret_cast<uintptr_t>(block_pairs) & 7u))
+    return PA_ERR_INVALID_ARG;
+  pa::CopyParams p;
+  p.dst_k = const_cast<void*>(device_view(dst_k_pool));
+  p.dst_v = const_cast<void*>(device_view(dst_v_pool));
+  p.src_k = device_view(src_k_pool);
+  p.src_v = device_view(src_v_pool);
+  p.pairs = static_cast<const int64_t*>(device_view(block_pairs));
+  if (!p.dst_k || !p.dst_v || !p.src_k || !p.src_v || !p.pairs) return PA_ERR_INVALID_ARG;
+  p.dev_err = dev_err;
+  p.n_pairs = n_pairs;
+  p.src_num_blocks = src_num_blocks;
+  p.dst_num_blocks = dst_num_blocks;
   p.block_bytes = bb;
   return cuda_status(pa::launch_copy_blocks(p, static_cast<cudaStream_t>(stream)));
 }

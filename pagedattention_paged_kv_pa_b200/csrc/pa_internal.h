@@ -73,12 +73,16 @@ struct ScatterParams {
 cudaError_t launch_reshape_and_cache(const ScatterParams& p, pa_dtype src_dt,
                                      pa_dtype cache_dt, cudaStream_t st);
 
+// Block copy from (src_k, src_v) to (dst_k, dst_v): the same pools for
+// copy-on-write, a device and a pinned host pool for swapping.
 struct CopyParams {
-  void* k_pool;
-  void* v_pool;
+  void* dst_k;
+  void* dst_v;
+  const void* src_k;
+  const void* src_v;
   const int64_t* pairs;
   int32_t* dev_err;
-  int n_pairs, num_blocks;
+  int n_pairs, src_num_blocks, dst_num_blocks;
   int64_t block_bytes;  // bytes of one block (all heads) in one pool
 };
 cudaError_t launch_copy_blocks(const CopyParams& p, cudaStream_t st);

@@ -111,6 +111,25 @@ def test_multi_query_decode_argument_errors_are_synchronous(B):
     assert _multi(B, 3, mb=512, ws=16, wsb=ws - 1) == B.PA_ERR_INVALID_ARG
 
 
+def test_swap_argument_errors_are_synchronous(B):
+    v = ctypes.c_void_p
+    L = B.lib
+    args = lambda **k: dict(dk=16, dv=16, sk=16, sv=16, pr=16, n=2, nkv=8, d=128, bs=16, sn=10,
+                            dn=10, dt=B.PA_BF16, **k)
+
+    def call(a):
+        return L.pa_swap_blocks(v(a["dk"]) if a["dk"] else None, v(a["dv"]), v(a["sk"]),
+                                v(a["sv"]), v(a["pr"]) if a["pr"] else None, a["n"], a["nkv"],
+                                a["d"], a["bs"], a["sn"], a["dn"], a["dt"], None, None)
+    assert call({**args(), "bs": 32}) == B.PA_ERR_UNSUPPORTED
+    assert call({**args(), "n": -1}) == B.PA_ERR_INVALID_ARG
+    assert call({**args(), "sn": 0}) == B.PA_ERR_INVALID_ARG
+    assert call({**args(), "n": 0}) == B.PA_OK
+    assert call({**args(), "dk": 0}) == B.PA_ERR_INVALID_ARG
+    assert call({**args(), "pr": 0}) == B.PA_ERR_INVALID_ARG
+    assert call({**args(), "sk": 24}) == B.PA_ERR_INVALID_ARG        # misaligned pool
+
+
 def test_cache_op_argument_errors_are_synchronous(B):
     v = ctypes.c_void_p
     L = B.lib

@@ -132,3 +132,61 @@ def test_copy_blocks_bad_pair_flagged(B, cuda_device):
     ko, vo = _raw(kp), _raw(vp)
     orc.copy_blocks(ko, vo, np.array([[1, 2]]), W.F16)
     assert np.array_equal(_raw(kg), ko)
+
+
+# ---------------------------------------------------------------------------
+# swap between a device pool and a pinned host pool
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", [W.BF16, W.FP8_E4M3, W.F32])
+@pytest.mark.parametrize("pairs_on_host", [False, True])
+def test_swap_round_trip_bit_exact(B, cuda_device, dt, pairs_on_host):
+    dev = cuda_device
+    n_kv, d = 8, 128
+    gk, gv = _pools(40, n_kv, d, dt, "cpu", seed=21)
+    gkd, gvd = gk.to(dev), gv.to(dev)
+    hk = torch.zeros((24,) + tuple(gk.shape[1:]), dtype=gk.dtype).pin_memory()
+    hv = torch.zeros_like(hk).pin_memory()
+    out_pairs = torch.tensor([[3, 0], [39, 23], [17, 5], [0, 11]], dtype=torch.int64)
+    pr = out_pairs.pin_memory() if pairs_on_host else out_pairs.to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.pa_swap_blocks(hk, hv, gkd, gvd, pr, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rk, rv = np.zeros_like(_raw(hk)), np.zeros_like(_raw(hv))
+    assert orc.swap_blocks(rk, rv, _raw(gk), _raw(gv), out_pairs.numpy(), dt) == 0
+    assert np.array_equal(_raw(hk), rk) and np.array_equal(_raw(hv), rv)
+    # back into other device blocks
+    back = torch.tensor([[0, 7], [23, 30], [5, 1], [11, 2]], dtype=torch.int64)
+    prb = back.pin_memory() if pairs_on_host else back.to(dev)
+    B.pa_swap_blocks(gkd, gvd, hk, hv, prb, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ek, ev = _raw(gk), _raw(gv)
+    assert orc.swap_blocks(ek, ev, rk, rv, back.numpy(), dt) == 0
+    assert np.array_equal(_raw(gkd), ek) and np.array_equal(_raw(gvd), ev)
+
+
+def test_swap_refuses_pageable_host_memory(B, cuda_device):
+    dev = cuda_device
+    gk, gv = (t.to(dev) for t in _pools(8, 2, 64, W.BF16, "cpu", seed=3))
+    hk = torch.zeros((4,) + tuple(gk.shape[1:]), dtype=gk.dtype)   # not pinned
+    hv = torch.zeros_like(hk)
+    pairs = torch.tensor([[1, 0]], dtype=torch.int64, device=dev)
+    with pytest.raises(B.PAError) as e:
+        B.pa_swap_blocks(hk, hv, gk, gv, pairs)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+    assert not hk.any() and not hv.any()
+
+
+def test_swap_out_of_range_ids_flagged(B, cuda_device):
+    dev = cuda_device
+    gk, gv = (t.to(dev) for t in _pools(8, 2, 64, W.BF16, "cpu", seed=5))
+    hk = torch.zeros((4,) + tuple(gk.shape[1:]), dtype=gk.dtype).pin_memory()
+    hv = torch.zeros_like(hk).pin_memory()
+    pairs = torch.tensor([[1, 0], [8, 1], [2, 4]], dtype=torch.int64, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.pa_swap_blocks(hk, hv, gk, gv, pairs, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 2  # PA_DEVERR_SLOT
+    assert torch.equal(hk[0], gk[1].cpu()) and not hk[1:].any()

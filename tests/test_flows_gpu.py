@@ -133,3 +133,82 @@ def test_shared_prefix_copy_on_write_flow(cuda_device):
         pos += n
     ref_private = orc.paged_decode(q, kp2, vp2, bt2, ctx, scale, W.BF16, W.BF16)
     assert np.array_equal(ref, ref_private)
+
+
+def test_preemption_by_swap_keeps_decode_bits(cuda_device):
+    """Sequences are preempted by swapping their blocks to a pinned host pool
+    ("vLLM explained", "KV cache 什麼時候可以被覆蓋": swap to the CPU when
+    memory runs short); new sequences take and overwrite the freed GPU blocks;
+    the preempted ones are swapped back into other GPU blocks and decode to
+    the same bits as before (attention depends only on logical contents)."""
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    dev = cuda_device
+    n_q, n_kv, d = 32, 8, 128
+    gpu = B.BlockAllocator(120, 16)
+    cpu = B.BlockAllocator(96, 16)
+    gen = torch.Generator(device="cpu").manual_seed(77)
+    shape = (120, n_kv, 16, d)
+    kp = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    vp = torch.zeros_like(kp)
+    hk = torch.zeros((96, n_kv, 16, d), dtype=torch.bfloat16).pin_memory()
+    hv = torch.zeros_like(hk).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    lens = [300, 17, 640, 129, 500, 64]
+
+    def write(alloc, seq, n, seed):
+        st, slots = alloc.append(seq, n)
+        assert st == 0
+        key, val = W.make_new_kv(n, n_kv, d, W.BF16, dev, seed=seed)
+        B.pa_reshape_and_cache(kp, vp, key, val, torch.tensor(slots, device=dev), dev_err=err)
+
+    for s, n in enumerate(lens):
+        write(gpu, s, n, 100 + s)
+    q = torch.randn(len(lens), n_q, d, generator=gen).to(torch.bfloat16).to(dev)
+
+    def decode(seqs):
+        mb = 48
+        bt = torch.full((len(seqs), mb), -1, dtype=torch.int32)
+        for r, s in enumerate(seqs):
+            t = gpu.block_table(s)
+            bt[r, :len(t)] = torch.tensor(t, dtype=torch.int32)
+        cl = torch.tensor([gpu.num_tokens(s) for s in seqs], dtype=torch.int32)
+        out = torch.empty(len(seqs), n_q, d, dtype=torch.bfloat16, device=dev)
+        B.pa_decode(out, q[seqs], kp, vp, bt.to(dev), cl.to(dev), 1 / np.sqrt(d), dev_err=err)
+        return out
+
+    before = decode(list(range(len(lens))))
+    # preempt sequences 0, 2, 4: host blocks for their tokens, copy out, free on the GPU
+    swapped = [0, 2, 4]
+    old_tables = {s: gpu.block_table(s) for s in swapped}
+    pairs = []
+    for s in swapped:
+        st, _ = cpu.append(s, gpu.num_tokens(s))
+        assert st == 0
+        pairs += list(zip(gpu.block_table(s), cpu.block_table(s)))
+    B.pa_swap_blocks(hk, hv, kp, vp, torch.tensor(pairs, dtype=torch.int64, device=dev),
+                     dev_err=err)
+    for s in swapped:
+        assert gpu.free_seq(s) == 0
+    # new sequences take the never-used blocks, then freed ones, overwriting
+    # them; they finish before the preempted sequences come back
+    reused = set()
+    for s in range(10, 14):
+        write(gpu, s, 200, 200 + s)
+        reused |= set(gpu.block_table(s))
+    assert reused & {b for t in old_tables.values() for b in t}
+    for s in range(10, 14):
+        assert gpu.free_seq(s) == 0
+    # swap the preempted sequences back in, into whatever blocks are free now
+    pairs = []
+    for s in swapped:
+        st, _ = gpu.append(s, cpu.num_tokens(s))
+        assert st == 0
+        pairs += list(zip(cpu.block_table(s), gpu.block_table(s)))
+        assert cpu.free_seq(s) == 0
+    B.pa_swap_blocks(kp, vp, hk, hv, torch.tensor(pairs, dtype=torch.int64).pin_memory(),
+                     dev_err=err)
+    after = decode(swapped)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert any(gpu.block_table(s) != old_tables[s] for s in swapped)
+    assert torch.equal(after, before[swapped])
