@@ -783,6 +783,115 @@ def run_spec_verify(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def run_shared_prefix(args, rank, world, local):
+    """Decode over the shared-prefix sampling workload (16 prompts x 4 samples,
+    each prompt's 2048+ token prefix in blocks its samples share), with
+    pa_decode_shared_prefix (each group's shared blocks read once for the
+    group) and, for comparison, plain pa_decode.  GB/s are reported on logical
+    bytes (every sequence's whole context) and on unique bytes (each shared
+    block once)."""
+    import torch
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist_init(world, "nccl")
+    inp, _ = W.make_shared_prefix_inputs(dev)
+    spec = inp.spec
+    ctx = inp.context_lens.cpu().numpy()
+    groups = B.prefix_groups(inp.block_tables, inp.context_lens, spec.n_q_heads,
+                             spec.n_kv_heads, spec.kv_dtype)
+    gdev = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in groups.items()}
+    out = torch.empty_like(inp.q)
+    mb = inp.block_tables.shape[1]
+    ws = B.alloc_decode_workspace(inp.q, mb)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    logical = W.decode_algorithmic_bytes(ctx, spec.n_q_heads, spec.n_kv_heads, spec.head_dim, 2, 2)
+    shared_tok = int(sum((len([m for m in row if m >= 0]) - 1) * nb * 16 for row, nb in
+                         zip(groups["members"].tolist(), groups["shared_blocks"].tolist())))
+    unique = logical - shared_tok * 2 * spec.n_kv_heads * spec.head_dim * 2
+
+    def call(shared):
+        if shared:
+            B.pa_decode_shared_prefix(out, inp.q, inp.k_pool, inp.v_pool, inp.block_tables,
+                                      inp.context_lens, inp.scale, gdev, workspace=ws,
+                                      dev_err=err)
+        else:
+            B.pa_decode(out, inp.q, inp.k_pool, inp.v_pool, inp.block_tables, inp.context_lens,
+                        inp.scale, workspace=ws, dev_err=err)
+
+    def timed(shared, K):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        for i in range(K):
+            # the unique K/V (210 MB) is not far above the 126 MB L2: flush it
+            # before each timed call
+            _l2_flush(dev)
+            evs[i][0].record()
+            call(shared)
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / K
+
+    for shared in (True, False):
+        for _ in range(max(args.warmup, 3)):
+            call(shared)
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    K = args.steps
+    barrier(world, dev)
+    ms = reduce_over_ranks(timed(True, K), "max", world, dev)
+    ms_plain = reduce_over_ranks(timed(False, K), "max", world, dev)
+    barrier(world, dev)
+    clocks = sampler.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+    peak, _ = hbm_peak()
+    line = {
+        "metric": METRIC, "value": round(logical * world / (ms / 1e3) / 1e9, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"shared-prefix sampling: 16 prompts x 4 samples, prompt 2048 + "
+                               f"U{{1..15}}, 0-512 divergent tokens, 32 q / 8 kv heads, bf16 "
+                               f"(sum {int(ctx.sum())} tokens, {inp.num_blocks} unique blocks, "
+                               f"{len(groups['members'])} groups)",
+                   "logical_bytes": int(logical), "unique_bytes": int(unique),
+                   "l2": "flushed (256 MB write) before every timed call",
+                   "parallelism": f"replicas x{world}"},
+        "unique_gbs": round(unique / (ms / 1e3) / 1e9, 1),
+        "roofline": {"bound": "hbm", "achieved": round(unique / (ms / 1e3) / 1e9, 1),
+                     "peak": peak, "unit": "GB/s",
+                     "frac": round(unique / (ms / 1e3) / 1e9 / peak, 4), "traffic": None,
+                     "kernel": "pa_decode_shared_prefix (group + per-sequence partition "
+                               "kernels + merge), on unique bytes"},
+        "plain_decode": {"us": round(ms_plain * 1e3, 2),
+                         "logical_gbs": round(logical / (ms_plain / 1e3) / 1e9, 1),
+                         "unique_gbs": round(unique / (ms_plain / 1e3) / 1e9, 1)},
+        "speedup_vs_plain_decode": round(ms_plain / ms, 3),
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+_FLUSH = {}
+
+
+def _l2_flush(dev):
+    """Write 256 MB (twice the L2) so that no K/V stays cached between calls."""
+    import torch
+    buf = _FLUSH.get(dev)
+    if buf is None:
+        buf = _FLUSH[dev] = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    buf.fill_(1)
+
+
 def run_swap(args, rank, world, local):
     """Swap preemption's data path: 4,096 blocks of the Llama-3-70B GQA layer
     (8 kv heads x 16 tokens x 128 dims, bf16, K and V: 256 MB) from the device
@@ -964,6 +1073,8 @@ def main(argv=None):
         run_alloc_host(args)
     elif args.workload == "swap_bf16":
         run_swap(args, rank, world, local)
+    elif args.workload == "shared_prefix_bf16":
+        run_shared_prefix(args, rank, world, local)
     else:
         run_ours(args, rank, world, local)
 

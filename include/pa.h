@@ -177,6 +177,62 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_pool, const vo
                           void* stream);
 
 /*
+ * pa_decode_shared_prefix -- pa_decode's result, reading each block that a
+ * group of sequences shares at the start of their tables once for the whole
+ * group: the samples of one prompt share its blocks ([P1] §三.2: parallel
+ * sampling forks share physical blocks; [P2] "帶來的好處"), so attention over
+ * the shared prefix is one pass over those K/V for all members' queries (one
+ * (member, head) pair per MMA column) instead of one pass per member.
+ *
+ * Group g has members group_members[g][0 .. group_width) (sequence indices;
+ * -1 pads) whose tables hold the same ids in their first
+ * group_shared_blocks[g] entries, all within every member's context;
+ * seq_group[s] is the group of sequence s or -1.  The group pass computes the
+ * context partitions (see pa_decode) that lie wholly inside a group's shared
+ * blocks, for every member at once; each sequence's own pass computes its
+ * other partitions; the merge is pa_decode's.  pa_prefix_groups builds these
+ * arrays from host copies of the block tables.
+ *
+ *   group_members, group_shared_blocks, seq_group  device int32 arrays
+ *   group_width  members per group; group_width x (n_q_heads / n_kv_heads)
+ *                must be <= 32
+ *   other arguments as pa_decode (same workspace size).
+ * n_groups == 0 gives pa_decode.  Supported: q_dtype F16 or BF16 when
+ * n_groups > 0.  Group arrays that break the contract above give wrong
+ * results, not memory errors: every index is range-checked on the device.
+ */
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
+                                  const void* v_pool, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, int block_size,
+                                  int n_q_heads, int n_kv_heads, int head_dim, int num_seqs,
+                                  int max_blocks_per_seq, int num_blocks, pa_dtype q_dtype,
+                                  pa_dtype kv_dtype, float k_scale, float v_scale,
+                                  const int32_t* group_members, const int32_t* group_shared_blocks,
+                                  const int32_t* seq_group, int n_groups, int group_width,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                                  void* stream);
+
+/*
+ * pa_prefix_groups -- host helper for pa_decode_shared_prefix: groups the
+ * sequences whose tables start with the same block (in index order, at most
+ * 32 / (n_q_heads / n_kv_heads) per group) and records how many leading
+ * blocks all members share, within their full blocks; groups sharing less
+ * than one whole partition, and single sequences, are dropped.
+ * *group_width_out is the largest group's size (the row stride of
+ * group_members_out).
+ *
+ *   block_tables, context_lens  host copies ([num_seqs][max_blocks_per_seq],
+ *                [num_seqs])
+ *   group_members_out  host int32 of num_seqs x 32 / G entries
+ *   group_shared_blocks_out, seq_group_out  host int32 [num_seqs]
+ */
+pa_status pa_prefix_groups(const int32_t* block_tables, const int32_t* context_lens,
+                           int num_seqs, int max_blocks_per_seq, int n_q_heads, int n_kv_heads,
+                           pa_dtype kv_dtype, int32_t* group_members_out,
+                           int32_t* group_shared_blocks_out, int32_t* seq_group_out,
+                           int* n_groups_out, int* group_width_out);
+
+/*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
  * memory and therefore have no workspace to pass: for example a plugin inside
  * a host program that owns all device memory and forbids cudaMalloc after

@@ -31,7 +31,7 @@ EXPORTS = (
     "pa_alloc_num_seqs", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes",
     "pa_decode_multi", "pa_alloc_set_prefix_caching", "pa_alloc_admit",
     "pa_alloc_append_tokens", "pa_alloc_cached_list", "pa_alloc_num_cached",
-    "pa_swap_blocks",
+    "pa_swap_blocks", "pa_decode_shared_prefix", "pa_prefix_groups",
 )
 
 
@@ -85,6 +85,9 @@ def _load() -> ctypes.CDLL:
     L.pa_alloc_num_free.argtypes = [P]
     L.pa_alloc_num_seqs.argtypes = [P]
     L.pa_swap_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    L.pa_decode_shared_prefix.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, F, F,
+                                          P, P, P, I, I, P, Z, P, P]
+    L.pa_prefix_groups.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
     L.pa_alloc_set_prefix_caching.argtypes = [P, I]
     L.pa_alloc_admit.argtypes = [P, I64, P, I, P, P]
     L.pa_alloc_append_tokens.argtypes = [P, I64, P, I, P]
@@ -185,6 +188,47 @@ def pa_decode_multi(out, q, k_pool, v_pool, block_tables, context_lens, scale, k
                                mb, num_blocks, dtype_code(q), dtype_code(k_pool), float(k_scale),
                                float(v_scale), _p(workspace), ws_bytes, _p(dev_err),
                                _stream(stream, q.device)), "pa_decode_multi")
+    return out
+
+
+def prefix_groups(block_tables, context_lens, n_q_heads: int, n_kv_heads: int, kv_dtype: int):
+    """Groups of sequences whose block tables start with the same blocks (from
+    host copies), as pa_decode_shared_prefix takes them: a dict with
+    members [n_groups, width], shared_blocks [n_groups], seq_group [num_seqs]
+    (int32 CPU tensors) and width."""
+    bt = block_tables.detach().cpu().contiguous().to(torch.int32)
+    cl = context_lens.detach().cpu().contiguous().to(torch.int32)
+    ns, mb = bt.shape
+    width = 32 // (n_q_heads // n_kv_heads)
+    members = torch.full((max(ns, 1), width), -1, dtype=torch.int32)
+    shared = torch.zeros(max(ns, 1), dtype=torch.int32)
+    seq_group = torch.full((max(ns, 1),), -1, dtype=torch.int32)
+    ng, w = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.pa_prefix_groups(_p(bt), _p(cl), ns, mb, n_q_heads, n_kv_heads, kv_dtype,
+                                _p(members), _p(shared), _p(seq_group), ctypes.byref(ng),
+                                ctypes.byref(w)), "pa_prefix_groups")
+    n, w = ng.value, w.value
+    flat = members.view(-1)[:n * w]
+    return {"members": flat.view(n, w).clone(), "shared_blocks": shared[:n].clone(),
+            "seq_group": seq_group[:ns].clone(), "width": w}
+
+
+def pa_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, context_lens, scale, groups,
+                            k_scale=1.0, v_scale=1.0, workspace=None, dev_err=None, stream=None):
+    """pa_decode's result with each group's shared prefix read once for the
+    group (groups as returned by prefix_groups, on any device)."""
+    if workspace is None:
+        workspace = alloc_decode_workspace(q, block_tables.shape[1])
+    dev = q.device
+    members = groups["members"].to(dev, torch.int32).contiguous()
+    shared = groups["shared_blocks"].to(dev, torch.int32).contiguous()
+    seq_group = groups["seq_group"].to(dev, torch.int32).contiguous()
+    a = _decode_args(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale,
+                     v_scale, workspace, dev_err, stream)
+    # pa_decode's arguments with the group arrays before the workspace
+    _check(lib.pa_decode_shared_prefix(*a[:18], _p(members), _p(shared), _p(seq_group),
+                                       members.shape[0], int(groups["width"]), *a[18:]),
+           "pa_decode_shared_prefix")
     return out
 
 

@@ -2,7 +2,9 @@
 // builds (and caches) TMA tensor maps over the KV pools, and queues the
 // kernels on the caller's stream.  No device memory is allocated here and no
 // call synchronises with the device.
+#include <algorithm>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "pa_internal.h"
@@ -178,7 +180,11 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
                                int head_dim, int num_seqs, int q_len, int max_blocks_per_seq,
                                int num_blocks, pa_dtype q_dtype, pa_dtype kv_dtype,
                                float k_scale, float v_scale, void* workspace,
-                               size_t workspace_bytes, int32_t* dev_err, void* stream) {
+                               size_t workspace_bytes, int32_t* dev_err, void* stream,
+                               const int32_t* grp_members = nullptr,
+                               const int32_t* grp_shared_blocks = nullptr,
+                               const int32_t* seq_group = nullptr, int n_groups = 0,
+                               int grp_width = 0) {
   DecodeShape s{n_q_heads, n_kv_heads, head_dim, num_seqs, max_blocks_per_seq, num_blocks,
                 pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   pa_status st = check_decode(s, block_size, q_dtype, kv_dtype);
@@ -227,14 +233,30 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
   p.n_parts_grid = n_grid;
   p.q_len = q_len;
   p.n_cg = n_cg;
+  p.grp_members = nullptr;
+  p.grp_shared_blocks = nullptr;
+  p.seq_group = nullptr;
+  p.grp_width = 0;
+  p.n_groups = n_groups;
+  p.n_seqs_all = num_seqs;
   CUtensorMap tmk, tmv;
   if (pa::decode_uses_tma(q_dtype, kv_dtype)) {
     if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
         !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv))
       return PA_ERR_CUDA;
   }
-  return cuda_status(pa::launch_decode_partitions(p, head_dim, q_dtype, kv_dtype, &tmk, &tmv,
-                                                  static_cast<cudaStream_t>(stream)));
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (n_groups > 0) {
+    // one launch: the groups' shared partitions, every member at once (one
+    // column per (member, head)), next to every sequence's other partitions
+    if ((int64_t)n_groups + num_seqs > 65535) return PA_ERR_UNSUPPORTED;
+    p.grp_members = grp_members;
+    p.grp_shared_blocks = grp_shared_blocks;
+    p.seq_group = seq_group;
+    p.grp_width = grp_width;
+    p.num_seqs = n_groups + num_seqs;  // grid z: groups, then sequences
+  }
+  return cuda_status(pa::launch_decode_partitions(p, head_dim, q_dtype, kv_dtype, &tmk, &tmv, cs));
 }
 
 pa_status pa_decode_partitions(void* out, const void* q, const void* k_pool, const void* v_pool,
@@ -319,6 +341,109 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_pool, const vo
   return decode_reduce_impl(out, context_lens, n_q_heads * q_len, head_dim, num_seqs,
                             max_blocks_per_seq, q_dtype, kv_dtype, v_scale, workspace,
                             workspace_bytes, stream);
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
+                                  const void* v_pool, const int32_t* block_tables,
+                                  const int32_t* context_lens, float scale, int block_size,
+                                  int n_q_heads, int n_kv_heads, int head_dim, int num_seqs,
+                                  int max_blocks_per_seq, int num_blocks, pa_dtype q_dtype,
+                                  pa_dtype kv_dtype, float k_scale, float v_scale,
+                                  const int32_t* group_members, const int32_t* group_shared_blocks,
+                                  const int32_t* seq_group, int n_groups, int group_width,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                                  void* stream) {
+  if (n_groups < 0) return PA_ERR_INVALID_ARG;
+  if (n_groups > 0) {
+    if (!group_members || !group_shared_blocks || !seq_group || group_width < 1)
+      return PA_ERR_INVALID_ARG;
+    if (q_dtype != PA_F16 && q_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+    if (n_kv_heads < 1 || n_q_heads % n_kv_heads != 0 ||
+        group_width * (n_q_heads / n_kv_heads) > 32 || n_groups > 65535)
+      return PA_ERR_UNSUPPORTED;
+  }
+  pa_status st = decode_parts_impl(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                                   block_size, n_q_heads, n_kv_heads, head_dim, num_seqs, 1,
+                                   max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                                   v_scale, workspace, workspace_bytes, dev_err, stream,
+                                   group_members, group_shared_blocks, seq_group, n_groups,
+                                   group_width);
+  if (st != PA_OK) return st;
+  return decode_reduce_impl(out, context_lens, n_q_heads, head_dim, num_seqs, max_blocks_per_seq,
+                            q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_prefix_groups(const int32_t* block_tables, const int32_t* context_lens,
+                           int num_seqs, int max_blocks_per_seq, int n_q_heads, int n_kv_heads,
+                           pa_dtype kv_dtype, int32_t* group_members_out,
+                           int32_t* group_shared_blocks_out, int32_t* seq_group_out,
+                           int* n_groups_out, int* group_width_out) {
+  if (!n_groups_out || !group_width_out || num_seqs < 0 || max_blocks_per_seq < 1 ||
+      n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads != 0 || !valid_dtype(kv_dtype))
+    return PA_ERR_INVALID_ARG;
+  const int G = n_q_heads / n_kv_heads;
+  if (G > 8) return PA_ERR_UNSUPPORTED;
+  const int W = 32 / G;  // members per group: 4 column groups of 8 (member, head) pairs
+  *n_groups_out = 0;
+  *group_width_out = W;
+  if (num_seqs == 0) return PA_OK;
+  if (!block_tables || !context_lens || !group_members_out || !group_shared_blocks_out ||
+      !seq_group_out)
+    return PA_ERR_INVALID_ARG;
+  const int part_blocks = pa::decode_part_tokens(kv_dtype) / 16;
+  std::vector<int> full(num_seqs);
+  for (int s = 0; s < num_seqs; s++) {
+    const int c = context_lens[s] < 0 ? 0 : context_lens[s];
+    full[s] = std::min(c / 16, max_blocks_per_seq);
+    seq_group_out[s] = -1;
+  }
+  // sequences whose first block is the same, in index order
+  std::unordered_map<int32_t, std::vector<int>> by_first;
+  std::vector<int32_t> firsts;
+  for (int s = 0; s < num_seqs; s++) {
+    if (full[s] < part_blocks) continue;  // shares no whole partition
+    const int32_t b = block_tables[(size_t)s * max_blocks_per_seq];
+    auto it = by_first.find(b);
+    if (it == by_first.end()) {
+      firsts.push_back(b);
+      by_first[b] = {s};
+    } else {
+      it->second.push_back(s);
+    }
+  }
+  std::vector<std::pair<std::vector<int>, int>> groups;  // (members, shared blocks)
+  for (int32_t b : firsts) {
+    const std::vector<int>& cand = by_first[b];
+    for (size_t c0 = 0; c0 < cand.size(); c0 += W) {
+      const size_t n = std::min(cand.size() - c0, (size_t)W);
+      if (n < 2) continue;
+      const int s0 = cand[c0];
+      int shared = full[s0];
+      for (size_t k = 1; k < n; k++) {
+        const int s = cand[c0 + k];
+        int m = 0;
+        const int lim = std::min(shared, full[s]);
+        while (m < lim && block_tables[(size_t)s * max_blocks_per_seq + m] ==
+                              block_tables[(size_t)s0 * max_blocks_per_seq + m])
+          m++;
+        shared = m;
+      }
+      if (shared < part_blocks) continue;
+      groups.emplace_back(std::vector<int>(cand.begin() + c0, cand.begin() + c0 + n), shared);
+    }
+  }
+  // rows as wide as the largest group, so the group pass has no empty columns
+  int w = 0;
+  for (auto& g : groups) w = std::max(w, (int)g.first.size());
+  for (size_t g = 0; g < groups.size(); g++) {
+    const auto& m = groups[g].first;
+    for (int k = 0; k < w; k++) group_members_out[g * w + k] = k < (int)m.size() ? m[k] : -1;
+    group_shared_blocks_out[g] = groups[g].second;
+    for (int s : m) seq_group_out[s] = (int)g;
+  }
+  *n_groups_out = (int)groups.size();
+  *group_width_out = groups.empty() ? W : w;
+  return PA_OK;
 }
 
 pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,

@@ -99,6 +99,19 @@ __device__ __forceinline__ size_t col_row(const DecodeParams& p, int seq, int kv
   return ((size_t)seq * p.q_len + i) * p.n_q + (size_t)kvh * p.group + (m - i * p.group);
 }
 
+// Group CTA of the shared-prefix decode: column c of column group cg is
+// head m % G of member m / G of group grp (m = 8cg + c); -1 for a column of an
+// unused member slot.  *member receives the member's sequence.
+__device__ __forceinline__ long long grp_col_row(const DecodeParams& p, int grp, int kvh, int cg,
+                                                 int c, int* member) {
+  const int m = 8 * cg + c, i = m / p.group;
+  int s = i < p.grp_width ? p.grp_members[(size_t)grp * p.grp_width + i] : -1;
+  if (s >= p.n_seqs_all) s = -1;  // not a sequence: the column is left out
+  *member = s;
+  if (s < 0) return -1;
+  return (long long)s * p.n_q + (long long)kvh * p.group + (m - i * p.group);
+}
+
 // Merge the consumer warps' (m, l, O) states held in shared memory and write
 // the partition result.  The CTA's nvc columns are "virtual columns"
 // vc = 8 gi + c of its column groups gi (group cg0 + gi of the sequence's
@@ -111,7 +124,7 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
                                                 float* Ls, float* Ms, int nthreads,
                                                 const DecodeParams& p, int seq, int kvh,
                                                 int cg0, int cpc2, int wpg, int nvc, int part,
-                                                int n_parts_seq) {
+                                                int n_parts_seq, int part_tokens, bool grp) {
   const int tid = threadIdx.x;
   if (tid < nvc) {
     const int gi = tid >> 3, c = tid & 7;
@@ -128,16 +141,33 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
     Ms[tid] = M;
   }
   __syncthreads();
+  // the row of a virtual column and how many partitions its sequence has
+  // (in a group CTA each column has its own member sequence)
+  auto target = [&](int vc, int& np) -> long long {
+    if (grp) {
+      int ms;
+      const long long r = grp_col_row(p, seq, kvh, cg0 + (vc >> 3), vc & 7, &ms);
+      if (r >= 0) {
+        const int c = max(0, min(p.context_lens[ms], p.max_blocks * 16));
+        np = (c + part_tokens - 1) / part_tokens;
+      }
+      return r;
+    }
+    np = n_parts_seq;
+    return (long long)col_row(p, seq, kvh, cg0 + (vc >> 3), vc & 7);
+  };
   for (int idx = tid; idx < nvc * D; idx += nthreads) {
     const int vc = idx / D, dd = idx % D;
     const int gi = vc >> 3, c = vc & 7;
+    int np = 1;
+    const long long row = target(vc, np);
+    if (row < 0) continue;
     float acc = 0.f;
     for (int ph = 0; ph < wpg; ++ph) {
       const int w = gi + cpc2 * ph;
       acc += wgt[w * 8 + c] * mo[(w * 8 + c) * D + dd];
     }
-    const size_t row = col_row(p, seq, kvh, cg0 + gi, c);
-    if (n_parts_seq == 1) {
+    if (np == 1) {
       const float L = Ls[vc];
       reinterpret_cast<OutT*>(p.out)[row * D + dd] =
           from_f32<OutT>(L > 0.f ? acc / L * p.out_mul : 0.f);
@@ -145,9 +175,12 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
       p.ws_o[(row * p.n_parts_max + part) * D + dd] = acc;
     }
   }
-  if (n_parts_seq > 1 && tid < nvc)
-    p.ws_ml[col_row(p, seq, kvh, cg0 + (tid >> 3), tid & 7) * p.n_parts_max + part] =
-        make_float2(Ms[tid], Ls[tid]);
+  if (tid < nvc) {
+    int np = 1;
+    const long long row = target(tid, np);
+    if (row >= 0 && np > 1)
+      p.ws_ml[row * p.n_parts_max + part] = make_float2(Ms[tid], Ls[tid]);
+  }
 }
 // ---------------------------------------------------------------------------
 // tensor-core engine: 16-bit caches (MMA in the cache's type) and fp8 caches
@@ -171,23 +204,53 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
-  const int part = blockIdx.x, seq = blockIdx.z;
+  const int part = blockIdx.x;
   const int G = p.group;
+  // shared-prefix decode: the first n_groups z-indices are groups, whose CTAs
+  // take every member's queries over the group's shared blocks (K/V through
+  // the first member's table, whole shared partitions only, no causal mask);
+  // the rest are sequences.
+  const bool grp = MQ && p.grp_members != nullptr && (int)blockIdx.z < p.n_groups;
+  const int seq = (MQ && p.grp_members && !grp) ? (int)blockIdx.z - p.n_groups : (int)blockIdx.z;
+  const int n_pairs = grp ? p.grp_width * G : G * p.q_len;  // (query or member, head) pairs
+  const int n_cg = (n_pairs + 7) >> 3;
   int kvh = blockIdx.y, cg0 = 0, cpc = 1, cpc2 = 1;
   if constexpr (MQ) {
-    const int nquad = (p.n_cg + 3) >> 2;
+    const int nquad = (p.n_cg + 3) >> 2;  // the grid's quads per kv head
     kvh = (int)blockIdx.y / nquad;
     cg0 = 4 * ((int)blockIdx.y - kvh * nquad);
-    cpc = min(4, p.n_cg - cg0);
+    if (cg0 >= n_cg) return;
+    cpc = min(4, n_cg - cg0);
     cpc2 = cpc == 1 ? 1 : (cpc == 2 ? 2 : 4);
   }
   const int wpg = kNW / cpc2;  // warps per column group
   // virtual columns in use: 8 per full group, the last group's remainder
-  const int nvc = MQ ? min(8 * cpc, G * p.q_len - 8 * cg0) : G;
-  const int ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
-                            threadIdx.x == 0 && part == 0 && blockIdx.y == 0);
+  const int nvc = MQ ? min(8 * cpc, n_pairs - 8 * cg0) : G;
   constexpr int kPart = L::kPart;
+  int tseq = seq, ctx;
+  if (grp) {
+    tseq = p.grp_members[(size_t)seq * p.grp_width];
+    const int sb = p.grp_shared_blocks[seq];
+    if (tseq < 0 || tseq >= p.n_seqs_all || sb < 0 || sb > p.max_blocks) {
+      if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+      return;
+    }
+    ctx = (sb * 16 / kPart) * kPart;
+    if (part * kPart >= ctx) return;
+  } else {
+    ctx = clamp_ctx(p.context_lens[seq], p.max_blocks * 16, p.dev_err,
+                    threadIdx.x == 0 && part == 0 && blockIdx.y == 0);
+  }
   const int tok0 = part * kPart;
+  if (!grp && p.seq_group && tok0 < ctx) {  // partitions a group launch computes
+    const int gi = p.seq_group[seq];
+    if (gi >= p.n_groups) {
+      if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+    } else if (gi >= 0) {
+      const int sb = p.grp_shared_blocks[gi];
+      if (sb >= 0 && sb <= p.max_blocks && part < sb * 16 / kPart) return;
+    }
+  }
   if (tok0 >= ctx) {
     if (part == 0) {  // empty context: all-zero output rows
       QT* out = reinterpret_cast<QT*>(p.out);
@@ -208,7 +271,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x < nblk) {
-    int id = p.block_tables[(size_t)seq * p.max_blocks + (tok0 >> 4) + threadIdx.x];
+    int id = p.block_tables[(size_t)tseq * p.max_blocks + (tok0 >> 4) + threadIdx.x];
     if (id < 0 || id >= p.num_blocks) {
       flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
       id = -1;
@@ -272,7 +335,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     // ------------------------------------------------------------ consumers
     const int gi = warp % cpc2, ph = warp / cpc2;  // column group, block phase
     const int cg = cg0 + gi;
-    const int ncols = MQ ? min(8, G * p.q_len - 8 * cg) : G;  // this warp's columns
+    const int ncols = MQ ? min(8, n_pairs - 8 * cg) : G;  // this warp's columns
     const bool active = !MQ || gi < cpc;
     // Q as the B operand (k = head dim, n = query head of the group); heads
     // beyond the group size are zero.  The fp8 path pairs MMA k-index
@@ -281,8 +344,17 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     // same pairing, which leaves the dot products unchanged.
     uint32_t qb[KS][2];
     {
-      const bool hv = g < ncols;
-      const QT* qrow = reinterpret_cast<const QT*>(p.q) + col_row(p, seq, kvh, cg, hv ? g : 0) * D;
+      bool hv = g < ncols;
+      size_t r = 0;
+      if (grp) {
+        int ms;
+        const long long gr = hv ? grp_col_row(p, seq, kvh, cg, g, &ms) : -1;
+        hv = gr >= 0;
+        r = hv ? (size_t)gr : 0;
+      } else {
+        r = col_row(p, seq, kvh, cg, hv ? g : 0);
+      }
+      const QT* qrow = reinterpret_cast<const QT*>(p.q) + r * D;
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         if constexpr (FP8) {
@@ -354,7 +426,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
         }
         if constexpr (MQ) {
           const int kb = tok0 + 16 * j;  // position of the block's first key
-          if (kb + 16 > lim_min) {
+          if (!grp && kb + 16 > lim_min) {  // (a group launch has no causal mask)
             const int k0 = kb + g, k1 = k0 + 8;
             if (k0 >= lim_a) x0 = -INFINITY;
             if (k0 >= lim_b) x1 = -INFINITY;
@@ -505,7 +577,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
   }
   __syncthreads();
   merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, cg0, cpc2, wpg, nvc,
-                         part, n_parts_seq);
+                         part, n_parts_seq, kPart, grp);
 }
 
 // ---------------------------------------------------------------------------
@@ -602,7 +674,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeP
   }
   __syncthreads();
   merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, 0, 1, kNW, G, part,
-                            n_parts_seq);
+                            n_parts_seq, kPart, false);
 }
 
 // ---------------------------------------------------------------------------
@@ -668,8 +740,8 @@ cudaError_t launch_mma_(const DecodeParams& p, const CUtensorMap* tmk, const CUt
 template <int D, bool FP8, bool Q_BF16>
 cudaError_t launch_mma(const DecodeParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
                        cudaStream_t st) {
-  return p.q_len > 1 ? launch_mma_<D, FP8, Q_BF16, true>(p, tmk, tmv, st)
-                     : launch_mma_<D, FP8, Q_BF16, false>(p, tmk, tmv, st);
+  return (p.q_len > 1 || p.grp_members) ? launch_mma_<D, FP8, Q_BF16, true>(p, tmk, tmv, st)
+                                        : launch_mma_<D, FP8, Q_BF16, false>(p, tmk, tmv, st);
 }
 
 template <int D>

@@ -40,6 +40,18 @@ struct DecodeParams {
   int n_parts_grid;  // partitions of max_blocks at this cache type's length
   int q_len;         // queries per sequence (1: decode; >1: multi-query decode)
   int n_cg;          // groups of 8 (query, head) columns per kv head
+  // shared-prefix decode: groups of sequences whose tables start with the
+  // same blocks.  grp_members [n_groups][grp_width] (-1: unused),
+  // grp_shared_blocks [n_groups], seq_group [num_seqs] (-1: none).  A group
+  // launch (grp_members set) computes the partitions wholly inside a group's
+  // shared blocks for all members; a per-sequence launch with seq_group set
+  // skips them.
+  const int32_t* grp_members;
+  const int32_t* grp_shared_blocks;
+  const int32_t* seq_group;
+  int grp_width;
+  int n_groups;     // for range checks of seq_group
+  int n_seqs_all;   // for range checks of grp_members (num_seqs is the grid)
 };
 
 struct ReduceParams {

@@ -264,6 +264,57 @@ def make_decode_inputs(spec: DecodeSpec, device="cpu", ctx: Optional[np.ndarray]
                         torch.from_numpy(ctx).to(device), scale, k_scale, v_scale)
 
 
+# Shared-prefix parallel sampling ("LLM inference optimization", §三.2: the
+# samples of a prompt share its blocks): 16 prompts x 4 samples, 32 q / 8 kv
+# heads, bf16; prompt 2048 + U{1..15} tokens (its full blocks shared by the 4
+# samples), then 0-512 divergent tokens per sample in private blocks.
+SHARED_PREFIX_BF16 = DecodeSpec("shared_prefix_bf16", 64, 32, 8, 128, BF16, BF16, "fixed",
+                                ((),), max_ctx=2048 + 15 + 512 + 16, seed=1004)
+
+
+def make_shared_prefix_inputs(device="cpu", n_prompts: int = 16, n_samples: int = 4,
+                              seed: int = 1004):
+    """Decode inputs whose sequences 4p .. 4p+3 share prompt p's full blocks.
+    Returns (DecodeInputs, groups) with groups[p] = the prompt's sample
+    indices and its number of shared full blocks."""
+    rng = _rng(seed)
+    plen = 2048 + rng.integers(1, 16, size=n_prompts)
+    div = rng.integers(0, 513, size=(n_prompts, n_samples))
+    B = BLOCK_SIZE
+    shared = [int(l) // B for l in plen]
+    ctx = np.array([int(plen[p] + div[p, s]) for p in range(n_prompts)
+                    for s in range(n_samples)], np.int32)
+    private = [-(-int(ctx[p * n_samples + s]) // B) - shared[p] for p in range(n_prompts)
+               for s in range(n_samples)]
+    num_blocks = sum(shared) + sum(private)
+    perm = rng.permutation(num_blocks).astype(np.int32)
+    spec = SHARED_PREFIX_BF16.scaled(num_seqs=n_prompts * n_samples)
+    mb = spec.max_blocks_per_seq
+    bt = np.full((n_prompts * n_samples, mb), -1, np.int32)
+    nxt = 0
+    groups = []
+    for p in range(n_prompts):
+        pref = perm[nxt:nxt + shared[p]]
+        nxt += shared[p]
+        members = []
+        for s in range(n_samples):
+            i = p * n_samples + s
+            bt[i, :shared[p]] = pref
+            k = private[i]
+            bt[i, shared[p]:shared[p] + k] = perm[nxt:nxt + k]
+            nxt += k
+            members.append(i)
+        groups.append((members, shared[p]))
+    gen = _torch_gen(device, seed)
+    pool_shape = (num_blocks, spec.n_kv_heads, B, spec.head_dim)
+    q = randn_as((spec.num_seqs, spec.n_q_heads, spec.head_dim), spec.q_dtype, device, gen)
+    k_pool = randn_as(pool_shape, spec.kv_dtype, device, gen)
+    v_pool = randn_as(pool_shape, spec.kv_dtype, device, gen)
+    inp = DecodeInputs(spec, q, k_pool, v_pool, torch.from_numpy(bt).to(device),
+                       torch.from_numpy(ctx).to(device), 1.0 / math.sqrt(spec.head_dim), 1.0, 1.0)
+    return inp, groups
+
+
 def make_multi_queries(inp: DecodeInputs, q_len: int, seed: int) -> torch.Tensor:
     """Queries [num_seqs, q_len, n_q, d] for multi-query decode over inp's cache
     (N(0,1) draws rounded to the query dtype)."""

@@ -5,7 +5,9 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "pa.h")
@@ -145,3 +147,35 @@ def test_cache_op_argument_errors_are_synchronous(B):
                             None) == B.PA_ERR_INVALID_ARG
     assert L.pa_copy_blocks(None, None, None, 0, 8, 128, 16, 10, B.PA_BF16, None,
                             None) == B.PA_OK
+
+
+def test_prefix_groups_from_host_tables(B):
+    # bf16 caches: 1024-token partitions = 64 blocks.  Sequences 0-3 start with
+    # block 7; 0-2 share 70 blocks, 3 leaves them after 64; 4 is alone; 5 starts
+    # with block 7 too but holds less than one partition; 6, 7 share 100 blocks.
+    mb = 110
+    bt = np.full((8, mb), -1, np.int32)
+    pre = np.arange(1000, 1000 + 100, dtype=np.int32)
+    pre[0] = 7
+    for s in (0, 1, 2, 3):
+        bt[s, :70] = pre[:70]
+    bt[3, 64:70] = np.arange(5000, 5006)
+    bt[4, :70] = np.arange(6000, 6070)
+    bt[5, :10] = pre[:10]
+    other = np.arange(8000, 8105, dtype=np.int32)
+    bt[6, :105] = other
+    bt[7, :100] = other[:100]
+    bt[7, 100:103] = [9000, 9001, 9002]
+    ctx = np.array([70 * 16, 70 * 16 - 5, 70 * 16, 70 * 16, 70 * 16, 150, 105 * 16, 103 * 16],
+                   np.int32)
+    g = B.prefix_groups(torch.from_numpy(bt), torch.from_numpy(ctx), 32, 8, B.PA_BF16)
+    assert g["width"] == 4
+    assert g["members"].tolist() == [[0, 1, 2, 3], [6, 7, -1, -1]]
+    # 1's context ends 5 tokens into its 70th block: 69 full blocks; 3 diverges at 64
+    assert g["shared_blocks"].tolist() == [64, 100]
+    assert g["seq_group"].tolist() == [0, 0, 0, 0, -1, -1, 1, 1]
+    # groups are at most 32 / G wide: with G = 8, 4 members
+    bt2 = np.tile(bt[6], (6, 1))
+    g2 = B.prefix_groups(torch.from_numpy(bt2), torch.full((6,), 1600, dtype=torch.int32),
+                         64, 8, B.PA_BF16)
+    assert g2["members"].tolist() == [[0, 1, 2, 3], [4, 5, -1, -1]]
