@@ -119,7 +119,7 @@ __device__ __forceinline__ long long grp_col_row(const DecodeParams& p, int grp,
 // w = gi + cpc2 * ph.  Plain decode: one group (cg0 = 0, cpc2 = 1) over all
 // kNW warps, nvc = G.  mo: [kNW][8][D], mm/ml/wgt: [kNW][8] (log2-domain max,
 // running sum, merge weight), Ls/Ms: [32].  Called by every thread of the CTA.
-template <int D, typename OutT>
+template <int D, typename OutT, bool MQ>
 __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml, float* wgt,
                                                 float* Ls, float* Ms, int nthreads,
                                                 const DecodeParams& p, int seq, int kvh,
@@ -144,6 +144,10 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
   // the row of a virtual column and how many partitions its sequence has
   // (in a group CTA each column has its own member sequence)
   auto target = [&](int vc, int& np) -> long long {
+    if constexpr (!MQ) {  // plain decode: the G heads of the kv head
+      np = n_parts_seq;
+      return ((long long)seq * p.n_q + (long long)kvh * p.group) + vc;
+    }
     if (grp) {
       int ms;
       const long long r = grp_col_row(p, seq, kvh, cg0 + (vc >> 3), vc & 7, &ms);
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
                     threadIdx.x == 0 && part == 0 && blockIdx.y == 0);
   }
   const int tok0 = part * kPart;
-  if (!grp && p.seq_group && tok0 < ctx) {  // partitions a group launch computes
+  if (MQ && !grp && p.seq_group && tok0 < ctx) {  // partitions the group CTAs compute
     const int gi = p.seq_group[seq];
     if (gi >= p.n_groups) {
       if (threadIdx.x == 0 && blockIdx.y == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
@@ -256,7 +260,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
       QT* out = reinterpret_cast<QT*>(p.out);
       for (int idx = threadIdx.x; idx < nvc * D; idx += kThreads) {
         const int vc = idx / D;
-        out[col_row(p, seq, kvh, cg0 + (vc >> 3), vc & 7) * D + idx % D] = from_f32<QT>(0.f);
+        const size_t row = MQ ? col_row(p, seq, kvh, cg0 + (vc >> 3), vc & 7)
+                              : (size_t)seq * p.n_q + (size_t)kvh * G + vc;
+        out[row * D + idx % D] = from_f32<QT>(0.f);
       }
     }
     return;
@@ -351,8 +357,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
         const long long gr = hv ? grp_col_row(p, seq, kvh, cg, g, &ms) : -1;
         hv = gr >= 0;
         r = hv ? (size_t)gr : 0;
-      } else {
+      } else if constexpr (MQ) {
         r = col_row(p, seq, kvh, cg, hv ? g : 0);
+      } else {
+        r = (size_t)seq * p.n_q + (size_t)kvh * G + (hv ? g : 0);
       }
       const QT* qrow = reinterpret_cast<const QT*>(p.q) + r * D;
 #pragma unroll
@@ -576,8 +584,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     }
   }
   __syncthreads();
-  merge_and_store<D, QT>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, cg0, cpc2, wpg, nvc,
-                         part, n_parts_seq, kPart, grp);
+  merge_and_store<D, QT, MQ>(mo, mm, ml, wgt, Ls, Ms, kThreads, p, seq, kvh, cg0, cpc2, wpg, nvc,
+                             part, n_parts_seq, kPart, grp);
 }
 
 // ---------------------------------------------------------------------------
@@ -673,8 +681,8 @@ __global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeP
     }
   }
   __syncthreads();
-  merge_and_store<D, float>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, 0, 1, kNW, G, part,
-                            n_parts_seq, kPart, false);
+  merge_and_store<D, float, false>(mo, mm, ml, wgt, Ls, Ms, kNW * 32, p, seq, kvh, 0, 1, kNW, G,
+                                   part, n_parts_seq, kPart, false);
 }
 
 // ---------------------------------------------------------------------------
