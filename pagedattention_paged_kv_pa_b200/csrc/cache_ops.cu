@@ -16,6 +16,9 @@ namespace {
 // "PagedAttention" items 1-4).
 template <typename SrcT, bool TO_FP8>
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(const ScatterParams p) {
+  // the attention kernel that follows may start its set-up now; it waits for
+  // this grid before it reads the cache
+  pdl_launch_dependents();
   constexpr int EPC = 16 / sizeof(SrcT);  // source elements per chunk
   const int cpr = p.head_dim / EPC;       // chunks per row
   const int64_t per_kv = (int64_t)p.num_tokens * p.n_kv * cpr;

@@ -32,6 +32,7 @@
 // per-tensor scales are applied to the scores and to the final output.  fp32
 // inputs use a CUDA-core path with fp32 arithmetic throughout.
 #include <type_traits>
+#include <utility>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -207,6 +208,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  // the merge kernel may be scheduled as this grid drains (it waits for it)
+  pdl_launch_dependents();
 
   const int part = blockIdx.x;
   const int G = p.group;
@@ -305,6 +308,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
       const uint64_t pol = l2_policy_evict_first();
+      // the cache may have been written by the kernel before this one (the
+      // step's slot write, launched ahead of us): wait for it before reading
+      pdl_wait();
       int issued = 0;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % kStages;
@@ -691,6 +697,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_simt_f32_kernel(const DecodeP
 // ---------------------------------------------------------------------------
 template <int D, typename OutT>
 __global__ void __launch_bounds__(256) decode_reduce_kernel(const ReduceParams r) {
+  pdl_wait();  // the partition results of the kernel before this one
   constexpr int VPL = D / 32;
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -734,6 +741,24 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream is still running (see pdl_wait).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int D, bool FP8, bool Q_BF16, bool MQ>
 cudaError_t launch_mma_(const DecodeParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv,
                         cudaStream_t st) {
@@ -741,8 +766,8 @@ cudaError_t launch_mma_(const DecodeParams& p, const CUtensorMap* tmk, const CUt
   static cudaError_t attr = set_smem(decode_mma_kernel<D, FP8, Q_BF16, MQ>, L::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   dim3 grid(p.n_parts_grid, p.n_kv * (MQ ? (p.n_cg + 3) / 4 : 1), p.num_seqs);
-  decode_mma_kernel<D, FP8, Q_BF16, MQ><<<grid, kThreads, L::kSmemBytes, st>>>(*tmk, *tmv, p);
-  return cudaGetLastError();
+  return launch_pdl(decode_mma_kernel<D, FP8, Q_BF16, MQ>, grid, dim3(kThreads), L::kSmemBytes,
+                    st, *tmk, *tmv, p);
 }
 
 template <int D, bool FP8, bool Q_BF16>
@@ -788,16 +813,11 @@ cudaError_t launch_decode_reduce(const ReduceParams& r, int D, pa_dtype out_dt,
                                  cudaStream_t st) {
   const int blocks = (r.num_seqs * r.n_q + 7) / 8;
   if (blocks == 0) return cudaSuccess;
-#define PA_RED(DD, T) decode_reduce_kernel<DD, T><<<blocks, 256, 0, st>>>(r)
-  if (out_dt == PA_F32) {
-    if (D == 64) PA_RED(64, float); else PA_RED(128, float);
-  } else if (out_dt == PA_BF16) {
-    if (D == 64) PA_RED(64, __nv_bfloat16); else PA_RED(128, __nv_bfloat16);
-  } else {
-    if (D == 64) PA_RED(64, __half); else PA_RED(128, __half);
-  }
+#define PA_RED(DD, T) launch_pdl(decode_reduce_kernel<DD, T>, dim3(blocks), dim3(256), 0, st, r)
+  if (out_dt == PA_F32) return D == 64 ? PA_RED(64, float) : PA_RED(128, float);
+  if (out_dt == PA_BF16) return D == 64 ? PA_RED(64, __nv_bfloat16) : PA_RED(128, __nv_bfloat16);
+  return D == 64 ? PA_RED(64, __half) : PA_RED(128, __half);
 #undef PA_RED
-  return cudaGetLastError();
 }
 
 }  // namespace pa

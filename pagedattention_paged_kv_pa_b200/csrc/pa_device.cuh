@@ -141,6 +141,17 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before the previous kernel in its stream has
+// finished; pdl_wait() blocks the calling thread until that kernel has
+// completed and its memory operations are visible.  pdl_launch_dependents()
+// lets the next such kernel start once every CTA of this grid has issued it
+// (or exited).  Without a preceding programmatic launch both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
