@@ -79,6 +79,7 @@ def test_decode_argument_errors_are_synchronous(B):
     assert _dec(B, q=24) == B.PA_ERR_INVALID_ARG                  # misaligned pointer
     assert _dec(B, mb=0) == B.PA_ERR_INVALID_ARG
     assert _dec(B, ns=0) == B.PA_OK                               # nothing to do
+    assert _dec(B, ns=65536) == B.PA_ERR_UNSUPPORTED              # beyond the grid's z
     # more than one partition needs a workspace of the advertised size
     ws = B.pa_decode_workspace_size(4, 8, 128, 512)
     assert ws > 0

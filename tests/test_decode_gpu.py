@@ -148,3 +148,28 @@ def test_full_size_sampled(B, cuda_device, spec):
     ref = P.oracle_decode(sub)
     gpu = out[pick].float().cpu().numpy().astype(np.float64)
     P.assert_close(gpu, ref, spec.q_dtype, spec.kv_dtype, f"{spec.name} sampled")
+
+
+@pytest.mark.parametrize("kv_dt", [W.BF16, W.FP8_E4M3])
+def test_long_contexts_many_partitions(B, cuda_device, kv_dt):
+    # 100,000 and 65,537 tokens: 98 / 65 partitions of 1024 tokens (16-bit) or
+    # 49 / 33 of 2048 (fp8) -- more partitions than a warp has lanes for the
+    # merge kernel to fold, and a ragged last block
+    ctx = np.array([100_000, 65_537, 5], np.int32)
+    spec = W.DecodeSpec("long", 3, 8, 2, 128, W.BF16, kv_dt, "fixed", (ctx,),
+                        max_ctx=100_016, pool_factor=1.05, seed=91)
+    _check(W.make_decode_inputs(spec, ctx=ctx), cuda_device, f"long contexts kv={kv_dt}")
+
+
+def test_largest_batch(B, cuda_device):
+    # 65,535 sequences (the grid's z limit), one kv head, contexts 0..40
+    n = 65_535
+    ctx = (np.arange(n) % 41).astype(np.int32)
+    spec = W.DecodeSpec("wide", n, 2, 1, 64, W.BF16, W.BF16, "fixed", (ctx,), max_ctx=48,
+                        pool_factor=1.0, seed=92)
+    inp = W.make_decode_inputs(spec, ctx=ctx)
+    gpu, err = P.run_decode(inp, cuda_device)
+    assert err == 0
+    ref = P.oracle_decode(inp)
+    P.assert_close(gpu, ref, W.BF16, W.BF16, "65,535 sequences")
+    assert np.all(gpu[ctx == 0] == 0)
