@@ -295,7 +295,8 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_pool, const 
  * 2^-24; larger magnitudes overflow), a restriction the bf16-cache variant
  * carries.  A block id outside [0, num_blocks) is flagged with
  * PA_DEVERR_BLOCK_ID and its keys read as zeros.  The output is written in
- * q_dtype.
+ * q_dtype.  PA_ERR_UNSUPPORTED also when num_blocks * n_kv_heads * 16 >= 2^31
+ * (the pools are addressed as that many rows of head_dim elements).
  */
 pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
                            const int32_t* block_tables, const int32_t* query_start_loc,

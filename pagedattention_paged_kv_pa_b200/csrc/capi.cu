@@ -461,6 +461,7 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
     return PA_ERR_INVALID_ARG;
   if (n_chunks > 65535 || n_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
   if ((int64_t)max_blocks_per_seq * 16 >= (int64_t(1) << 30)) return PA_ERR_UNSUPPORTED;
+  if ((int64_t)num_blocks * n_kv_heads * 16 >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
   if (q_dtype != PA_BF16 || (kv_dtype != PA_BF16 && kv_dtype != PA_FP8_E4M3))
     return PA_ERR_UNSUPPORTED;
   if (!(scale == scale) || (kv_dtype == PA_FP8_E4M3 && !(k_scale > 0.f && v_scale > 0.f)))
@@ -489,8 +490,12 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
   p.max_blocks = max_blocks_per_seq;
   p.num_blocks = num_blocks;
   p.max_chunk_len = max_chunk_len;
-  return cuda_status(
-      pa::launch_prefill(p, kv_dtype, k_pool, v_pool, static_cast<cudaStream_t>(stream)));
+  CUtensorMap tmk{}, tmv{};
+  if (fp8 && (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
+              !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv)))
+    return PA_ERR_CUDA;
+  return cuda_status(pa::launch_prefill(p, kv_dtype, k_pool, v_pool, &tmk, &tmv,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 pa_status pa_reshape_and_cache(void* k_pool, void* v_pool, const void* key, const void* value,

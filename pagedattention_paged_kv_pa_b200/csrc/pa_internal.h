@@ -110,7 +110,9 @@ struct PrefillParams {
   float out_mul;
   int n_q, n_kv, group, n_chunks, max_blocks, num_blocks, max_chunk_len;
 };
+// tmk / tmv: TMA maps over the fp8 pools (the decode kernel's; unused for bf16)
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k_pool,
-                           const void* v_pool, cudaStream_t st);
+                           const void* v_pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                           cudaStream_t st);
 
 }  // namespace pa

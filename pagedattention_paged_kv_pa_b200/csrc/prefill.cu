@@ -48,20 +48,29 @@ namespace {
 constexpr int D = 128;       // head dim
 constexpr int BM = 128;      // rows per CTA tile
 constexpr int BN = 128;      // keys per tile
-constexpr int kThreads = 288;
-constexpr int kSoftmaxWarps = 4, kMmaWarp = 8;  // warps 4-7 convert K/V
+constexpr int kSoftmaxWarps = 4, kMmaWarp = 8, kLoadWarp = 9;  // warps 4-7 convert K/V
 // TMEM columns: S[2] (2 x 128 fp32), O (128 fp32), P[2] (2 x 64 columns of f16 pairs)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 
-// shared-memory map (offsets from a 1024-aligned base)
+// shared-memory map (offsets from a 1024-aligned base).  With an fp8 cache a
+// tenth warp brings each tile's raw K and V rows into a 2-stage ring by TMA
+// (16 KiB each), and the converters widen them from there; two V stages then
+// fit instead of four.
 constexpr int kOpBytes = BM * D * 2;  // one 128x128 16-bit operand = 32 KiB
-constexpr int kKStages = 2, kVStages = 4;
-constexpr int kQOff = 0;
-constexpr int kKOff = kQOff + kOpBytes;              // K stages
-constexpr int kVOff = kKOff + kKStages * kOpBytes;   // V stages
-constexpr int kBarOff = kVOff + kVStages * kOpBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;
+constexpr int kRawBytes = BN * D;     // one tile's fp8 K (or V) rows = 16 KiB
+constexpr int kKStages = 2, kMaxVStages = 4, kRawStages = 2;
+template <bool FP8>
+struct Layout {
+  static constexpr int kThreads = FP8 ? 320 : 288;
+  static constexpr int kVStages = FP8 ? 2 : 4;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kOpBytes;             // K stages
+  static constexpr int kVOff = kKOff + kKStages * kOpBytes;  // V stages
+  static constexpr int kRawOff = kVOff + kVStages * kOpBytes;  // raw fp8 K, V stages
+  static constexpr int kBarOff = kRawOff + (FP8 ? kRawStages * 2 * kRawBytes : 0);
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+};
 
 // 128x128 16-bit operand with the 128-byte swizzle: 128-byte rows of 64
 // elements in two 16 KiB halves; chunk = 8 consecutive elements of a row
@@ -171,7 +180,8 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 struct Bars {
-  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kMaxVStages], v_empty[kMaxVStages];
+  uint64_t raw_full[kRawStages], raw_empty[kRawStages];
   uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2], done;
   uint32_t tmem_base;
   int abort_flag;
@@ -196,9 +206,13 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 }
 
 template <bool FP8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const void* __restrict__ k_pool,
-                      const void* __restrict__ v_pool) {
+                      const void* __restrict__ v_pool, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
+  using LY = Layout<FP8>;
+  constexpr int kVStages = LY::kVStages;
+  constexpr int kQOff = LY::kQOff, kKOff = LY::kKOff, kVOff = LY::kVOff, kBarOff = LY::kBarOff;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars* B = reinterpret_cast<Bars*>(smem + kBarOff);
@@ -232,6 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&B->v_full[s], 128);
       mbar_init(&B->v_empty[s], 1);
+    }
+    for (int s = 0; s < kRawStages; ++s) {
+      mbar_init(&B->raw_full[s], 1);
+      mbar_init(&B->raw_empty[s], 128);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B->s_full[s], 1);
@@ -317,6 +335,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&B->done);
       mbar_wait(&B->done, 0);
     }
+  } else if (warp == kLoadWarp) {
+    // ------------------------------------------------- raw fp8 tiles by TMA
+    // (this warp exists only with an fp8 cache) Lane m < 8 loads block m of
+    // tile t: its 16 K rows and 16 V rows of 128 bytes, one box each, into raw
+    // stage t % 2 with the 128-byte swizzle.  Blocks past the context and
+    // out-of-range ids are not loaded; the converters zero those keys.
+    if constexpr (FP8) {
+      const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
+      if (lane == 0) {
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
+      }
+      int issued = 0;
+      for (int t = 0; t < nkt; ++t) {
+        const int rs = t % kRawStages;
+        // the stage is free once every converter has read tile t-2 out of it
+        // (each lane waits, so each load it issues is ordered after those reads)
+        const bool ok = t < kRawStages ||
+                        (wait_or_abort(&B->raw_empty[rs], ((t - kRawStages) / kRawStages) & 1,
+                                       B, p.dev_err) &&
+                         !aborted(B));
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int blk = t * 8 + lane;
+        const int phys = (lane < 8 && blk * 16 < ctx) ? __ldg(&bt[blk]) : -1;
+        const bool valid = phys >= 0 && phys < p.num_blocks;
+        const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+        if (lane == 0) mbar_arrive_expect_tx(&B->raw_full[rs], __popc(vm) * 2u * 16u * D);
+        __syncwarp();
+        if (valid) {
+          uint8_t* dst = smem + LY::kRawOff + rs * 2 * kRawBytes + lane * 16 * D;
+          const int y = (phys * p.n_kv + kvh) * 16;  // row of the pool's [token rows][D] view
+          tma_load_2d(dst, &tmk, &B->raw_full[rs], 0, y);
+          tma_load_2d(dst + kRawBytes, &tmv, &B->raw_full[rs], 0, y);
+        }
+        issued = t + 1;
+      }
+      // loads still in flight when the CTA gives up land before it exits
+      if (lane == 0)
+        for (int t = max(0, issued - kRawStages); t < issued; ++t)
+          mbar_wait(&B->raw_full[t % kRawStages], (t / kRawStages) & 1);
+    }
   } else if (warp >= kSoftmaxWarps) {
     // ------------------------------------------------------------ converters
     const int ct = tid - kSoftmaxWarps * 32;  // 0..127
@@ -338,9 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = j & 1, sv = j % kVStages;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + sv * kOpBytes;
-      // bulk-prefetch tile j+1's K and V blocks into L2, so that the loads of
-      // the next tile hit L2 instead of HBM
-      if (j + 1 < nkt && ct < 16) {
+      // bf16: bulk-prefetch tile j+1's K and V blocks into L2, so that the
+      // loads of the next tile hit L2 instead of HBM; fp8: wait for the raw tile
+      bool raw_stop = false;
+      const int rs = j % kRawStages;
+      const uint8_t* raw = smem + LY::kRawOff + rs * 2 * kRawBytes;
+      if constexpr (FP8)
+        raw_stop = !wait_or_abort(&B->raw_full[rs], (j / kRawStages) & 1, B, p.dev_err);
+      if (!FP8 && j + 1 < nkt && ct < 16) {
         const int blk = (j + 1) * 8 + (ct & 7);
         const int phys = blk * 16 < ctx ? __ldg(&bt[blk]) : -1;
         if (phys >= 0 && phys < p.num_blocks)
@@ -370,6 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int phys = id_cur[FP8 ? m : (m >> 1)];
             if (phys < 0 || phys >= p.num_blocks) {
               if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+            } else if constexpr (FP8) {
+              if (!raw_stop) {  // row kib of block m in the swizzled raw stage
+                const uint32_t ro = m * 16 * D + swz128(kib * 128 + cc * 16);
+                kr[u] = *reinterpret_cast<const uint4*>(raw + ro);
+                vr[u] = *reinterpret_cast<const uint4*>(raw + kRawBytes + ro);
+              }
             } else {
               const size_t off = (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
               kr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
@@ -378,9 +448,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (g0 == 0) {  // the K stage is free once S(j-2) is done, the V stage once
-                        // O += P V of tile j-4 is
-          bool stop = j >= kKStages &&
-                      !wait_or_abort(&B->k_empty[s], ((j - kKStages) / kKStages) & 1, B, p.dev_err);
+                        // O += P V of tile j - kVStages is
+          if constexpr (FP8) mbar_arrive(&B->raw_empty[rs]);  // raw tile j read
+          bool stop = raw_stop || (j >= kKStages && !wait_or_abort(&B->k_empty[s],
+                                                                   ((j - kKStages) / kKStages) & 1,
+                                                                   B, p.dev_err));
           stop = stop || (j >= kVStages &&
                           !wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1, B,
                                          p.dev_err));
@@ -596,23 +668,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <bool FP8>
 cudaError_t launch_tc(const PrefillParams& p, const void* k_pool, const void* v_pool,
-                      cudaStream_t st) {
+                      const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st) {
+  using LY = Layout<FP8>;
   static cudaError_t attr = cudaFuncSetAttribute(
-      prefill_tc_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      prefill_tc_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   const int QT = BM / p.group;
   dim3 grid((p.max_chunk_len + QT - 1) / QT, p.n_kv, p.n_chunks);
-  prefill_tc_kernel<FP8><<<grid, kThreads, kSmemBytes, st>>>(p, k_pool, v_pool);
+  prefill_tc_kernel<FP8>
+      <<<grid, LY::kThreads, LY::kSmemBytes, st>>>(p, k_pool, v_pool, *tmk, *tmv);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k_pool,
-                           const void* v_pool, cudaStream_t st) {
+                           const void* v_pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                           cudaStream_t st) {
   if (p.n_chunks == 0) return cudaSuccess;
-  return kv_dt == PA_FP8_E4M3 ? launch_tc<true>(p, k_pool, v_pool, st)
-                              : launch_tc<false>(p, k_pool, v_pool, st);
+  return kv_dt == PA_FP8_E4M3 ? launch_tc<true>(p, k_pool, v_pool, tmk, tmv, st)
+                              : launch_tc<false>(p, k_pool, v_pool, tmk, tmv, st);
 }
 
 }  // namespace pa
