@@ -454,6 +454,7 @@ def run_mixed(args, rank, world, local):
     pout = torch.empty_like(pinp.q)
     mb = dinp.block_tables.shape[1]
     ws = B.alloc_decode_workspace(dinp.q, mb)
+    pws = B.alloc_prefill_workspace(pinp.k_pool, pinp.block_tables)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     s_dec = torch.cuda.current_stream(dev)
     s_pre = torch.cuda.Stream(dev)
@@ -481,8 +482,8 @@ def run_mixed(args, rank, world, local):
             ev[0].record(s_pre)
         B.pa_prefill_paged(pout, pinp.q, pinp.k_pool, pinp.v_pool, pinp.block_tables,
                            pinp.query_start_loc, pinp.context_lens, pinp.scale,
-                           pspec.chunk_len, pinp.k_scale, pinp.v_scale, dev_err=err,
-                           stream=s_pre)
+                           pspec.chunk_len, pinp.k_scale, pinp.v_scale, workspace=pws,
+                           dev_err=err, stream=s_pre)
         if ev is not None:
             ev[1].record(s_pre)
 

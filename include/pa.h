@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 1
+#define PA_ABI_VERSION 2
 
 typedef enum {
     PA_OK = 0,
@@ -297,14 +297,30 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_pool, const 
  * PA_DEVERR_BLOCK_ID and its keys read as zeros.  The output is written in
  * q_dtype.  PA_ERR_UNSUPPORTED also when num_blocks * n_kv_heads * 16 >= 2^31
  * (the pools are addressed as that many rows of head_dim elements).
+ *
+ *   workspace      NULL, or device memory of at least
+ *                  pa_prefill_workspace_size(n_chunks, n_kv_heads, head_dim,
+ *                  max_blocks_per_seq, block_size) bytes, 16-byte aligned,
+ *                  owned by the caller and free for this call's duration.
+ * With NULL every query tile widens the K/V it reads to f16 itself.  With a
+ * workspace a first kernel widens each chunk's history once (per kv head)
+ * into it, and the tensor-core kernel streams the f16 operands from there;
+ * every query tile of a chunk shares them.  The results are identical up to
+ * the order of the fp32 accumulation (the same f16 operands either way).
+ * PA_ERR_INVALID_ARG if the workspace is too small or misaligned;
+ * PA_ERR_UNSUPPORTED if n_chunks * n_kv_heads * (max_blocks_per_seq * 16
+ * rounded up to 128) >= 2^31.
  */
+size_t pa_prefill_workspace_size(int n_chunks, int n_kv_heads, int head_dim,
+                                 int max_blocks_per_seq, int block_size);
 pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
                            const int32_t* block_tables, const int32_t* query_start_loc,
                            const int32_t* context_lens, float scale, int block_size,
                            int n_q_heads, int n_kv_heads, int head_dim, int n_chunks,
                            int max_chunk_len, int max_blocks_per_seq, int num_blocks,
                            pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale,
-                           float v_scale, int32_t* dev_err, void* stream);
+                           float v_scale, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_err, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* Slot write and copy-on-write block copy                                    */

@@ -32,6 +32,7 @@ EXPORTS = (
     "pa_decode_multi", "pa_alloc_set_prefix_caching", "pa_alloc_admit",
     "pa_alloc_append_tokens", "pa_alloc_cached_list", "pa_alloc_num_cached",
     "pa_swap_blocks", "pa_decode_shared_prefix", "pa_prefix_groups",
+    "pa_prefill_workspace_size",
 )
 
 
@@ -62,7 +63,9 @@ def _load() -> ctypes.CDLL:
     L.pa_decode_noalloc.restype = I
     L.pa_decode_noalloc_scratch_bytes.restype = Z
     L.pa_prefill_paged.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, F, F,
-                                   P, P]
+                                   P, Z, P, P]
+    L.pa_prefill_workspace_size.argtypes = [I, I, I, I, I]
+    L.pa_prefill_workspace_size.restype = Z
     L.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, F, P, P]
     L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
     for fn in ("pa_decode", "pa_decode_partitions", "pa_decode_reduce", "pa_prefill_paged",
@@ -283,18 +286,35 @@ def pa_decode_reduce(out, context_lens, max_blocks_per_seq, kv_dtype, v_scale=1.
 # prefill
 # --------------------------------------------------------------------------
 
+def pa_prefill_workspace_size(n_chunks: int, n_kv_heads: int, head_dim: int,
+                              max_blocks_per_seq: int, block_size: int = 16) -> int:
+    return lib.pa_prefill_workspace_size(n_chunks, n_kv_heads, head_dim, max_blocks_per_seq,
+                                         block_size)
+
+
+def alloc_prefill_workspace(k_pool: torch.Tensor, block_tables: torch.Tensor) -> torch.Tensor:
+    """Workspace for pa_prefill_paged over these chunks' block tables."""
+    num_blocks, n_kv, bs, d = k_pool.shape
+    n = pa_prefill_workspace_size(block_tables.shape[0], n_kv, d, block_tables.shape[1], bs)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=k_pool.device)
+
+
 def pa_prefill_paged(out, q, k_pool, v_pool, block_tables, query_start_loc, context_lens,
-                     scale, max_chunk_len, k_scale=1.0, v_scale=1.0, dev_err=None,
-                     stream=None):
+                     scale, max_chunk_len, k_scale=1.0, v_scale=1.0, workspace=None,
+                     dev_err=None, stream=None):
+    """workspace: None (the attention kernel widens K/V itself) or a device
+    buffer of pa_prefill_workspace_size bytes (widened once per chunk)."""
     _contig(out, q, k_pool, v_pool, block_tables, query_start_loc, context_lens)
     total_q, n_q, d = q.shape
     num_blocks, n_kv, bs, _ = k_pool.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.pa_prefill_paged(_p(out), _p(q), _p(k_pool), _p(v_pool), _p(block_tables),
                                 _p(query_start_loc), _p(context_lens), float(scale), bs, n_q,
                                 n_kv, d, context_lens.shape[0], int(max_chunk_len),
                                 block_tables.shape[1], num_blocks, dtype_code(q),
                                 dtype_code(k_pool), float(k_scale), float(v_scale),
-                                _p(dev_err), _stream(stream, q.device)), "pa_prefill_paged")
+                                _p(workspace), ws_bytes, _p(dev_err),
+                                _stream(stream, q.device)), "pa_prefill_paged")
     return out
 
 

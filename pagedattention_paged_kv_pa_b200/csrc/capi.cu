@@ -446,13 +446,24 @@ pa_status pa_prefix_groups(const int32_t* block_tables, const int32_t* context_l
   return PA_OK;
 }
 
+size_t pa_prefill_workspace_size(int n_chunks, int n_kv_heads, int head_dim,
+                                 int max_blocks_per_seq, int block_size) {
+  if (n_chunks < 0 || n_kv_heads < 1 || head_dim != 128 || max_blocks_per_seq < 1 ||
+      block_size != 16)
+    return 0;
+  // K and V: f16 [n_chunks][n_kv][stage_rows][head_dim]
+  return 2 * (size_t)n_chunks * n_kv_heads * pa::prefill_stage_rows(max_blocks_per_seq) *
+         head_dim * 2;
+}
+
 pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const void* v_pool,
                            const int32_t* block_tables, const int32_t* query_start_loc,
                            const int32_t* context_lens, float scale, int block_size,
                            int n_q_heads, int n_kv_heads, int head_dim, int n_chunks,
                            int max_chunk_len, int max_blocks_per_seq, int num_blocks,
                            pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
-                           int32_t* dev_err, void* stream) {
+                           void* workspace, size_t workspace_bytes, int32_t* dev_err,
+                           void* stream) {
   if (block_size != 16 || head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads != 0) return PA_ERR_INVALID_ARG;
   const int G = n_q_heads / n_kv_heads;
@@ -490,11 +501,27 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
   p.max_blocks = max_blocks_per_seq;
   p.num_blocks = num_blocks;
   p.max_chunk_len = max_chunk_len;
+  p.stage_rows = static_cast<int>(pa::prefill_stage_rows(max_blocks_per_seq));
   CUtensorMap tmk{}, tmv{};
-  if (fp8 && (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
-              !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv)))
+  if (workspace != nullptr) {
+    // the history of every chunk is widened once into the workspace; both fp8
+    // operands widen exactly there, so V needs no 2^-8 fold
+    if (!aligned16(workspace) ||
+        workspace_bytes < pa_prefill_workspace_size(n_chunks, n_kv_heads, head_dim,
+                                                    max_blocks_per_seq, block_size))
+      return PA_ERR_INVALID_ARG;
+    const uint64_t rows = (uint64_t)n_chunks * n_kv_heads * p.stage_rows;
+    if (rows >= (uint64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    p.out_mul = fp8 ? v_scale : 1.f;
+    const uint16_t* kst = static_cast<const uint16_t*>(workspace);
+    if (!get_map(kst, rows, 128, 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, &tmk) ||
+        !get_map(kst + rows * 128, rows, 128, 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, &tmv))
+      return PA_ERR_CUDA;
+  } else if (fp8 && (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
+                     !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv))) {
     return PA_ERR_CUDA;
-  return cuda_status(pa::launch_prefill(p, kv_dtype, k_pool, v_pool, &tmk, &tmv,
+  }
+  return cuda_status(pa::launch_prefill(p, kv_dtype, k_pool, v_pool, &tmk, &tmv, workspace,
                                         static_cast<cudaStream_t>(stream)));
 }
 

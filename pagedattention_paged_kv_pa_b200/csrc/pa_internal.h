@@ -109,10 +109,15 @@ struct PrefillParams {
   float scale_log2;
   float out_mul;
   int n_q, n_kv, group, n_chunks, max_blocks, num_blocks, max_chunk_len;
+  int stage_rows;  // workspace rows per (chunk, kv head): max_blocks * 16 rounded up to 128
 };
-// tmk / tmv: TMA maps over the fp8 pools (the decode kernel's; unused for bf16)
+// Without a workspace the attention kernel widens K/V itself (tmk / tmv: TMA
+// maps over the fp8 pools, the decode kernel's; unused for bf16).  With one,
+// a first pass widens every chunk's history into it (K rows, then V rows, f16
+// [n_chunks][n_kv][stage_rows][128]) and tmk / tmv map its two halves.
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k_pool,
                            const void* v_pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                           cudaStream_t st);
+                           void* workspace, cudaStream_t st);
+size_t prefill_stage_rows(int max_blocks);
 
 }  // namespace pa

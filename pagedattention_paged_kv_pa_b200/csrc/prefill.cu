@@ -48,27 +48,38 @@ namespace {
 constexpr int D = 128;       // head dim
 constexpr int BM = 128;      // rows per CTA tile
 constexpr int BN = 128;      // keys per tile
-constexpr int kSoftmaxWarps = 4, kMmaWarp = 8, kLoadWarp = 9;  // warps 4-7 convert K/V
+constexpr int kSoftmaxWarps = 4;
 // TMEM columns: S[2] (2 x 128 fp32), O (128 fp32), P[2] (2 x 64 columns of f16 pairs)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 
-// shared-memory map (offsets from a 1024-aligned base).  With an fp8 cache a
-// tenth warp brings each tile's raw K and V rows into a 2-stage ring by TMA
-// (16 KiB each), and the converters widen them from there; two V stages then
-// fit instead of four.
+// Where the K/V operands come from:
+//   kWidenBf16 / kWidenFp8: warps 4-7 read the tile's rows through the block
+//     table and widen them to f16 in shared memory (with an fp8 cache a tenth
+//     warp first brings the raw rows into a 2-stage ring by TMA);
+//   kStaged: the chunk's history was widened once into an f16 workspace by
+//     prefill_widen_kernel (all query tiles of a chunk and kv head share it),
+//     and a TMA warp streams ready operands; there are no converter warps.
+enum Mode : int { kWidenBf16 = 0, kWidenFp8 = 1, kStaged = 2 };
+
+// shared-memory map (offsets from a 1024-aligned base)
 constexpr int kOpBytes = BM * D * 2;  // one 128x128 16-bit operand = 32 KiB
 constexpr int kRawBytes = BN * D;     // one tile's fp8 K (or V) rows = 16 KiB
-constexpr int kKStages = 2, kMaxVStages = 4, kRawStages = 2;
-template <bool FP8>
+constexpr int kMaxKStages = 3, kMaxVStages = 4, kRawStages = 2;
+template <int MODE>
 struct Layout {
-  static constexpr int kThreads = FP8 ? 320 : 288;
-  static constexpr int kVStages = FP8 ? 2 : 4;
+  static constexpr bool kStagedOps = MODE == kStaged;
+  static constexpr bool kRawRing = MODE == kWidenFp8;
+  static constexpr int kMmaWarp = kStagedOps ? 4 : 8;
+  static constexpr int kLoadWarp = kStagedOps ? 5 : 9;  // none for kWidenBf16
+  static constexpr int kThreads = kStagedOps ? 192 : (kRawRing ? 320 : 288);
+  static constexpr int kKStages = kStagedOps ? 3 : 2;
+  static constexpr int kVStages = kStagedOps ? 3 : (kRawRing ? 2 : 4);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kOpBytes;             // K stages
   static constexpr int kVOff = kKOff + kKStages * kOpBytes;  // V stages
   static constexpr int kRawOff = kVOff + kVStages * kOpBytes;  // raw fp8 K, V stages
-  static constexpr int kBarOff = kRawOff + (FP8 ? kRawStages * 2 * kRawBytes : 0);
+  static constexpr int kBarOff = kRawOff + (kRawRing ? kRawStages * 2 * kRawBytes : 0);
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
@@ -119,7 +130,6 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void conv_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // barrier over the 128 converter threads that also ORs a flag across them
 __device__ __forceinline__ bool conv_bar_or(bool v) {
   uint32_t r;
@@ -180,7 +190,7 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 struct Bars {
-  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kMaxVStages], v_empty[kMaxVStages];
+  uint64_t k_full[kMaxKStages], k_empty[kMaxKStages], v_full[kMaxVStages], v_empty[kMaxVStages];
   uint64_t raw_full[kRawStages], raw_empty[kRawStages];
   uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2], done;
   uint32_t tmem_base;
@@ -205,13 +215,20 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return pack2<false>(f.x, f.y);
 }
 
-template <bool FP8>
-__global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
+// tmk / tmv: with kWidenFp8 maps over the fp8 pools ([token rows][128]
+// bytes, 16 x 128-byte boxes); with kStaged maps over the f16 workspace
+// ([rows][128] f16, 64 x 128-element boxes); unused with kWidenBf16
+template <int MODE>
+__global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const void* __restrict__ k_pool,
                       const void* __restrict__ v_pool, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
-  using LY = Layout<FP8>;
-  constexpr int kVStages = LY::kVStages;
+  using LY = Layout<MODE>;
+  constexpr bool FP8 = MODE == kWidenFp8;
+  constexpr int kKStages = LY::kKStages, kVStages = LY::kVStages;
+  constexpr int kMmaWarp = LY::kMmaWarp, kLoadWarp = LY::kLoadWarp;
+  // stage "full" barriers: a TMA transaction count (staged) or the 128 converters
+  constexpr uint32_t kFullCount = LY::kStagedOps ? 1 : 128;
   constexpr int kQOff = LY::kQOff, kKOff = LY::kKOff, kVOff = LY::kVOff, kBarOff = LY::kBarOff;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -240,11 +257,11 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kKStages; ++s) {
-      mbar_init(&B->k_full[s], 128);
+      mbar_init(&B->k_full[s], kFullCount);
       mbar_init(&B->k_empty[s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&B->v_full[s], 128);
+      mbar_init(&B->v_full[s], kFullCount);
       mbar_init(&B->v_empty[s], 1);
     }
     for (int s = 0; s < kRawStages; ++s) {
@@ -300,20 +317,20 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
       const uint32_t aQ = sbase + kQOff;
       bool ok = true;
       for (int j = 0; j <= nkt && ok; ++j) {
-        if (j < nkt) {  // S(j) = Q K(j)^T
-          const int s = j & 1;
-          ok = wait_or_abort(&B->k_full[s], (j >> 1) & 1, B, p.dev_err);
+        if (j < nkt) {  // S(j) = Q K(j)^T into TMEM buffer j % 2
+          const int s = j & 1, sk = j % kKStages;
+          ok = wait_or_abort(&B->k_full[sk], (j / kKStages) & 1, B, p.dev_err);
           if (ok && j >= 2) ok = wait_or_abort(&B->s_empty[s], ((j - 2) >> 1) & 1, B, p.dev_err);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t bK = sbase + kKOff + s * kOpBytes;
+          const uint32_t bK = sbase + kKOff + sk * kOpBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
             tc_mma(tS + s * BN, smem_desc(aQ + off), smem_desc(bK + off), idesc, kk > 0);
           }
           tc_commit(&B->s_full[s]);
-          tc_commit(&B->k_empty[s]);  // the K stage is free once S(j) is done
+          tc_commit(&B->k_empty[sk]);  // the K stage is free once S(j) is done
         }
         if (j >= 1) {  // O += P(j-1) V(j-1), P from TMEM
           const int jp = j - 1, b = jp & 1, sv = jp % kVStages;
@@ -336,12 +353,49 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
       mbar_wait(&B->done, 0);
     }
   } else if (warp == kLoadWarp) {
-    // ------------------------------------------------- raw fp8 tiles by TMA
-    // (this warp exists only with an fp8 cache) Lane m < 8 loads block m of
-    // tile t: its 16 K rows and 16 V rows of 128 bytes, one box each, into raw
-    // stage t % 2 with the 128-byte swizzle.  Blocks past the context and
-    // out-of-range ids are not loaded; the converters zero those keys.
-    if constexpr (FP8) {
+    if constexpr (LY::kStagedOps) {
+      // --------------------------------------- f16 operands from the workspace
+      // Tile j of this chunk and kv head is rows row0 + 128 j .. + 127 of the
+      // workspace; each operand is two 64-column boxes (its two 16 KiB halves,
+      // 128-byte swizzled), counted on the stage's full barrier.
+      if (lane == 0) {
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
+        const int row0 = (c * p.n_kv + kvh) * p.stage_rows;
+        int issued_k = 0, issued_v = 0;
+        for (int j = 0; j < nkt; ++j) {
+          const int sk = j % kKStages, sv = j % kVStages;
+          if (j >= kKStages && !(wait_or_abort(&B->k_empty[sk], ((j - kKStages) / kKStages) & 1,
+                                               B, p.dev_err) &&
+                                 !aborted(B)))
+            break;
+          uint8_t* kd = smem + kKOff + sk * kOpBytes;
+          mbar_arrive_expect_tx(&B->k_full[sk], kOpBytes);
+          tma_load_2d(kd, &tmk, &B->k_full[sk], 0, row0 + j * BN);
+          tma_load_2d(kd + kOpBytes / 2, &tmk, &B->k_full[sk], 64, row0 + j * BN);
+          issued_k = j + 1;
+          if (j >= kVStages && !(wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1,
+                                               B, p.dev_err) &&
+                                 !aborted(B)))
+            break;
+          uint8_t* vd = smem + kVOff + sv * kOpBytes;
+          mbar_arrive_expect_tx(&B->v_full[sv], kOpBytes);
+          tma_load_2d(vd, &tmv, &B->v_full[sv], 0, row0 + j * BN);
+          tma_load_2d(vd + kOpBytes / 2, &tmv, &B->v_full[sv], 64, row0 + j * BN);
+          issued_v = j + 1;
+        }
+        // loads still in flight when the CTA gives up land before it exits
+        for (int t = max(0, issued_k - kKStages); t < issued_k; ++t)
+          mbar_wait(&B->k_full[t % kKStages], (t / kKStages) & 1);
+        for (int t = max(0, issued_v - kVStages); t < issued_v; ++t)
+          mbar_wait(&B->v_full[t % kVStages], (t / kVStages) & 1);
+      }
+    } else if constexpr (FP8) {
+      // ----------------------------------------------- raw fp8 tiles by TMA
+      // Lane m < 8 loads block m of tile t: its 16 K rows and 16 V rows of
+      // 128 bytes, one box each, into raw stage t % 2 with the 128-byte
+      // swizzle.  Blocks past the context and out-of-range ids are not
+      // loaded; the converters zero those keys.
       const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
       if (lane == 0) {
         prefetch_tensormap(&tmk);
@@ -378,6 +432,7 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
     }
   } else if (warp >= kSoftmaxWarps) {
     // ------------------------------------------------------------ converters
+    if constexpr (!LY::kStagedOps) {
     const int ct = tid - kSoftmaxWarps * 32;  // 0..127
     const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
     const int kv_es = FP8 ? 1 : 2;
@@ -394,7 +449,7 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
     load_ids(0, id_cur);
     if (nkt > 1) load_ids(1, id_nxt);
     for (int j = 0; j < nkt; ++j) {
-      const int s = j & 1, sv = j % kVStages;
+      const int s = j % kKStages, sv = j % kVStages;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + sv * kOpBytes;
       // bf16: bulk-prefetch tile j+1's K and V blocks into L2, so that the
@@ -502,6 +557,7 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
       if (j + 2 < nkt) load_ids(j + 2, id_nxt);  // a whole tile ahead of its first use
     }
   conv_done:;
+    }
   } else {
     // ------------------------------------------------------------ softmax
     const int r = tid;  // row = TMEM lane
@@ -666,16 +722,79 @@ __global__ void __launch_bounds__(Layout<FP8>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------- widen pass
+// Writes keys 0 .. round_up(ctx_c, 128) - 1 of chunk c's history for kv head
+// h as f16 rows of the workspace: K to kst[(c n_kv + h) stage_rows + key][d],
+// V likewise to vst.  Keys at or past the context, and the keys of a block
+// whose id is out of range (flagged PA_DEVERR_BLOCK_ID), are written as
+// zeros, so the attention kernel reads finite values everywhere.  Both fp8
+// operands widen exactly (code x 1); bf16 converts to f16 as in the widening
+// kernel.  One CTA per 128-key tile; 16-byte loads and stores, a warp covering
+// whole stored rows.
 template <bool FP8>
+__global__ void __launch_bounds__(256)
+    prefill_widen_kernel(const PrefillParams p, const void* __restrict__ k_pool,
+                         const void* __restrict__ v_pool, uint16_t* __restrict__ kst,
+                         uint16_t* __restrict__ vst) {
+  const int t = blockIdx.x, kvh = blockIdx.y, c = blockIdx.z;
+  const int ctx = p.context_lens[c];
+  if (ctx < 0 || ctx > p.max_blocks * 16) return;  // the attention kernel flags it
+  const int k0 = t * BN;
+  if (k0 >= ctx) return;
+  const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
+  constexpr int kES = FP8 ? 1 : 2;        // bytes per stored element
+  constexpr int kCh = D * kES / 16;       // 16-byte chunks per stored row
+  const size_t row0 = ((size_t)c * p.n_kv + kvh) * p.stage_rows + k0;
+  for (int idx = threadIdx.x; idx < BN * kCh; idx += blockDim.x) {
+    const int r = idx / kCh, cc = idx % kCh;
+    const int key = k0 + r;
+    uint4 kr = make_uint4(0, 0, 0, 0), vr = make_uint4(0, 0, 0, 0);
+    if (key < ctx) {
+      const int phys = __ldg(&bt[key >> 4]);
+      if (phys < 0 || phys >= p.num_blocks) {
+        if ((key & 15) == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+      } else {
+        const size_t off =
+            (((size_t)phys * p.n_kv + kvh) * 16 + (key & 15)) * (D * kES) + (size_t)cc * 16;
+        kr = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
+        vr = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
+      }
+    }
+    uint4* kd = reinterpret_cast<uint4*>(kst + (row0 + r) * D);
+    uint4* vd = reinterpret_cast<uint4*>(vst + (row0 + r) * D);
+    if constexpr (FP8) {  // 16 codes -> 16 f16 (elements 16 cc .. 16 cc + 15)
+      const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w}, vw[4] = {vr.x, vr.y, vr.z, vr.w};
+      uint32_t kh[8], vh[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
+        kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
+        vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
+        vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
+      }
+      kd[2 * cc] = make_uint4(kh[0], kh[1], kh[2], kh[3]);
+      kd[2 * cc + 1] = make_uint4(kh[4], kh[5], kh[6], kh[7]);
+      vd[2 * cc] = make_uint4(vh[0], vh[1], vh[2], vh[3]);
+      vd[2 * cc + 1] = make_uint4(vh[4], vh[5], vh[6], vh[7]);
+    } else {
+      kd[cc] = make_uint4(bf16x2_to_f16x2(kr.x), bf16x2_to_f16x2(kr.y), bf16x2_to_f16x2(kr.z),
+                          bf16x2_to_f16x2(kr.w));
+      vd[cc] = make_uint4(bf16x2_to_f16x2(vr.x), bf16x2_to_f16x2(vr.y), bf16x2_to_f16x2(vr.z),
+                          bf16x2_to_f16x2(vr.w));
+    }
+  }
+}
+
+template <int MODE>
 cudaError_t launch_tc(const PrefillParams& p, const void* k_pool, const void* v_pool,
                       const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st) {
-  using LY = Layout<FP8>;
+  using LY = Layout<MODE>;
   static cudaError_t attr = cudaFuncSetAttribute(
-      prefill_tc_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmemBytes);
+      prefill_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   const int QT = BM / p.group;
   dim3 grid((p.max_chunk_len + QT - 1) / QT, p.n_kv, p.n_chunks);
-  prefill_tc_kernel<FP8>
+  prefill_tc_kernel<MODE>
       <<<grid, LY::kThreads, LY::kSmemBytes, st>>>(p, k_pool, v_pool, *tmk, *tmv);
   return cudaGetLastError();
 }
@@ -684,10 +803,26 @@ cudaError_t launch_tc(const PrefillParams& p, const void* k_pool, const void* v_
 
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k_pool,
                            const void* v_pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                           cudaStream_t st) {
+                           void* workspace, cudaStream_t st) {
   if (p.n_chunks == 0) return cudaSuccess;
-  return kv_dt == PA_FP8_E4M3 ? launch_tc<true>(p, k_pool, v_pool, tmk, tmv, st)
-                              : launch_tc<false>(p, k_pool, v_pool, tmk, tmv, st);
+  const bool fp8 = kv_dt == PA_FP8_E4M3;
+  if (workspace == nullptr)
+    return fp8 ? launch_tc<kWidenFp8>(p, k_pool, v_pool, tmk, tmv, st)
+               : launch_tc<kWidenBf16>(p, k_pool, v_pool, tmk, tmv, st);
+  uint16_t* kst = static_cast<uint16_t*>(workspace);
+  uint16_t* vst = kst + (size_t)p.n_chunks * p.n_kv * p.stage_rows * D;
+  const dim3 grid(p.stage_rows / BN, p.n_kv, p.n_chunks);
+  if (fp8)
+    prefill_widen_kernel<true><<<grid, 256, 0, st>>>(p, k_pool, v_pool, kst, vst);
+  else
+    prefill_widen_kernel<false><<<grid, 256, 0, st>>>(p, k_pool, v_pool, kst, vst);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_tc<kStaged>(p, k_pool, v_pool, tmk, tmv, st);
+}
+
+size_t prefill_stage_rows(int max_blocks) {
+  return ((size_t)max_blocks * 16 + BN - 1) / BN * BN;
 }
 
 }  // namespace pa

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(B):
 def test_library_needs_no_cuda_driver_to_load(B):
     out = subprocess.run(["ldd", B.LIB_PATH], capture_output=True, text=True).stdout
     assert "libcuda.so" not in out  # driver entry points are fetched at run time
-    assert B.lib.pa_abi_version() == 1
+    assert B.lib.pa_abi_version() == 2
 
 
 def test_status_strings(B):
@@ -180,3 +180,34 @@ def test_prefix_groups_from_host_tables(B):
     g2 = B.prefix_groups(torch.from_numpy(bt2), torch.full((6,), 1600, dtype=torch.int32),
                          64, 8, B.PA_BF16)
     assert g2["members"].tolist() == [[0, 1, 2, 3], [4, 5, -1, -1]]
+
+
+def _pre(B, **kw):
+    a = dict(out=16, q=16, k=16, v=16, bt=16, qsl=16, cl=16, scale=0.1, bs=16, nq=8, nkv=2,
+             d=128, nc=3, mcl=64, mb=5, nb=10, qdt=B.PA_BF16, kvdt=B.PA_FP8_E4M3, ks=1.0,
+             vs=1.0, ws=None, wsb=0, err=None, st=None)
+    a.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return B.lib.pa_prefill_paged(v(a["out"]), v(a["q"]), v(a["k"]), v(a["v"]), v(a["bt"]),
+                                  v(a["qsl"]), v(a["cl"]), a["scale"], a["bs"], a["nq"],
+                                  a["nkv"], a["d"], a["nc"], a["mcl"], a["mb"], a["nb"],
+                                  a["qdt"], a["kvdt"], a["ks"], a["vs"], v(a["ws"]), a["wsb"],
+                                  v(a["err"]), v(a["st"]))
+
+
+def test_prefill_workspace_size_and_refusals(B):
+    # K and V, f16, per (chunk, kv head): max_blocks * 16 keys rounded up to 128 rows
+    assert B.pa_prefill_workspace_size(3, 2, 128, 5) == 2 * 3 * 2 * 128 * 128 * 2
+    assert B.pa_prefill_workspace_size(3, 2, 128, 8) == 2 * 3 * 2 * 128 * 128 * 2
+    assert B.pa_prefill_workspace_size(3, 2, 128, 9) == 2 * 3 * 2 * 256 * 128 * 2
+    assert B.pa_prefill_workspace_size(0, 2, 128, 9) == 0
+    assert B.pa_prefill_workspace_size(3, 2, 64, 9) == 0     # head_dim 128 only
+    assert B.pa_prefill_workspace_size(3, 2, 128, 9, 32) == 0
+    need = B.pa_prefill_workspace_size(3, 2, 128, 5)
+    # none of these reach a launch, so they are safe without a GPU
+    assert _pre(B, ws=4096, wsb=need - 16) == B.PA_ERR_INVALID_ARG   # too small
+    assert _pre(B, ws=4104, wsb=need) == B.PA_ERR_INVALID_ARG        # misaligned
+    assert _pre(B, d=64) == B.PA_ERR_UNSUPPORTED
+    assert _pre(B, nq=6, nkv=4) == B.PA_ERR_INVALID_ARG
+    assert _pre(B, nb=1 << 27, nkv=2) == B.PA_ERR_UNSUPPORTED        # pool rows >= 2^31
+    assert _pre(B, nc=0) == B.PA_OK                                   # nothing to do
