@@ -70,16 +70,22 @@ template <int MODE>
 struct Layout {
   static constexpr bool kStagedOps = MODE == kStaged;
   static constexpr bool kRawRing = MODE == kWidenFp8;
-  static constexpr int kMmaWarp = kStagedOps ? 4 : 8;
-  static constexpr int kLoadWarp = kStagedOps ? 5 : 9;  // none for kWidenBf16
-  static constexpr int kThreads = kStagedOps ? 192 : (kRawRing ? 320 : 288);
+  // staged: each row's softmax is split over two warps (8 softmax warps)
+  static constexpr bool kSplitSoftmax = kStagedOps;
+  static constexpr int kSoftWarps = kSplitSoftmax ? 8 : 4;
+  static constexpr int kMmaWarp = 8;
+  static constexpr int kLoadWarp = 9;  // none for kWidenBf16
+  static constexpr int kThreads = (kStagedOps || kRawRing) ? 320 : 288;
   static constexpr int kKStages = kStagedOps ? 3 : 2;
-  static constexpr int kVStages = kStagedOps ? 3 : (kRawRing ? 2 : 4);
+  static constexpr int kVStages = kStagedOps ? 2 : (kRawRing ? 2 : 4);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kOpBytes;             // K stages
   static constexpr int kVOff = kKOff + kKStages * kOpBytes;  // V stages
   static constexpr int kRawOff = kVOff + kVStages * kOpBytes;  // raw fp8 K, V stages
-  static constexpr int kBarOff = kRawOff + (kRawRing ? kRawStages * 2 * kRawBytes : 0);
+  // split softmax: row maxima of the two halves [2 parities][2 halves][BM],
+  // then the halves' row sums [2][BM]
+  static constexpr int kRedOff = kRawOff + (kRawRing ? kRawStages * 2 * kRawBytes : 0);
+  static constexpr int kBarOff = kRedOff + (kSplitSoftmax ? 6 * BM * 4 : 0);
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
@@ -129,6 +135,17 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// named barrier `id` over `n` threads that also ORs a flag across them
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %3, 0;\n\t"
+      "bar.red.or.pred p, %1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(n), "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
 }
 // barrier over the 128 converter threads that also ORs a flag across them
 __device__ __forceinline__ bool conv_bar_or(bool v) {
@@ -270,8 +287,8 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B->s_full[s], 1);
-      mbar_init(&B->s_empty[s], 128);
-      mbar_init(&B->p_full[s], 128);
+      mbar_init(&B->s_empty[s], LY::kSoftWarps * 32);
+      mbar_init(&B->p_full[s], LY::kSoftWarps * 32);
       mbar_init(&B->pv_done[s], 1);
     }
     mbar_init(&B->done, 1);
@@ -430,7 +447,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         for (int t = max(0, issued - kRawStages); t < issued; ++t)
           mbar_wait(&B->raw_full[t % kRawStages], (t / kRawStages) & 1);
     }
-  } else if (warp >= kSoftmaxWarps) {
+  } else if (warp >= LY::kSoftWarps) {
     // ------------------------------------------------------------ converters
     if constexpr (!LY::kStagedOps) {
     const int ct = tid - kSoftmaxWarps * 32;  // 0..127
@@ -557,6 +574,167 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       if (j + 2 < nkt) load_ids(j + 2, id_nxt);  // a whole tile ahead of its first use
     }
   conv_done:;
+    }
+  } else if constexpr (LY::kSplitSoftmax) {
+    // ------------------------------------------- softmax, two warps per row
+    // Warps w and w + 4 share rows 32 (w % 4) .. + 31 (the TMEM lanes warp
+    // w % 4 may access): the first takes keys 0-63 of every tile and O
+    // columns 0-63, the second keys 64-127 and O columns 64-127.  The row max
+    // of a tile is combined through shared memory at a named barrier over the
+    // 256 softmax threads, which also ORs their failure flags so that all of
+    // them leave the loop at the same barrier; the row sum is combined once at
+    // the end.  Each thread does half a row's exponentials, and two warps per
+    // sub-partition hide each other's latencies.
+    const int q4 = warp & 3, hh = warp >> 2;
+    const int r = q4 * 32 + lane;  // row = TMEM lane
+    const int i = i0 + r / G, g = r % G;
+    const bool row_valid = i < L;
+    const int lim = H + i;  // last visible key
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    float* red_max = reinterpret_cast<float*>(smem + LY::kRedOff);  // [2][2][BM]
+    float* red_sum = red_max + 4 * BM;                              // [2][BM]
+    const float sl = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool fail = false;  // warp-uniform
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j & 1;
+      fail = __any_sync(0xffffffffu,
+                        fail || !wait_or_abort(&B->s_full[s], (j >> 1) & 1, B, p.dev_err));
+      tc_fence_after();
+      const int kbase = j * BN + hh * 64;  // first key of this half
+      const uint32_t tSrow = tS + lane_base + s * BN + hh * 64;
+      const bool full = __all_sync(0xffffffffu, row_valid && kbase + 63 <= lim) && sl > 0.f;
+      float mx = -INFINITY;
+      if (!fail) {  // pass 1: this half's max
+        float x[64];
+        tmem_ld32(tSrow, x);
+        tmem_ld32(tSrow + 32, x + 32);
+        tmem_wait_ld();
+        if (full) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, x[e]);
+          mx *= sl;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const bool vis = !row_valid || (kbase + e <= lim);
+            mx = fmaxf(mx, vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
+          }
+        }
+      }
+      red_max[((j & 1) * 2 + hh) * BM + r] = mx;
+      if (named_bar_or(2, LY::kSoftWarps * 32, fail || aborted(B))) {
+        fail = true;
+        break;
+      }
+      mx = fmaxf(mx, red_max[((j & 1) * 2 + (hh ^ 1)) * BM + r]);
+      // O and l are rescaled lazily: only when the max grew by more than 2^8;
+      // both halves of a row take the same decision
+      const float m_new = fmaxf(m_used, mx);
+      const bool rescale = m_new > m_used + kRescaleLog2;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = exp2f(m_used - m_new);  // 0 on the first tile
+        l *= alpha;
+        m_used = m_new;
+      }
+      // pass 2: P = 2^(s*scale - m) as f16 pairs
+      float rs = 0.f;
+      uint32_t pk[32];
+      const float neg_m = -m_used;
+      {
+        float x[64];
+        tmem_ld32(tSrow, x);
+        tmem_ld32(tSrow + 32, x + 32);
+        tmem_wait_ld();
+        if (full) {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float a = fast_exp2(fmaf(x[e], sl, neg_m));
+            const float bb = fast_exp2(fmaf(x[e + 1], sl, neg_m));
+            rs += a + bb;
+            pk[e / 2] = pack2<false>(a, bb);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const int k0 = kbase + e;
+            const float v0 = row_valid ? (k0 <= lim ? x[e] * sl : -INFINITY) : 0.f;
+            const float v1 = row_valid ? (k0 + 1 <= lim ? x[e + 1] * sl : -INFINITY) : 0.f;
+            const float a = fast_exp2(v0 + neg_m), bb = fast_exp2(v1 + neg_m);
+            rs += a + bb;
+            pk[e / 2] = pack2<false>(a, bb);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&B->s_empty[s]);  // S buffer s may be overwritten by S(j+2)
+      l += rs;
+      const int b = j & 1;
+      // P buffer b is free once O += P V of tile j-2 has completed
+      if (j >= 2)
+        fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[b], ((j - 2) >> 1) & 1, B,
+                                                      p.dev_err));
+      // O (this half's columns) is rescaled, rarely, once O += P V of tile j-1
+      // has completed
+      if (!fail && j >= 1 && __any_sync(0xffffffffu, rescale)) {
+        fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[b ^ 1], ((j - 1) >> 1) & 1, B,
+                                                      p.dev_err));
+        if (!fail) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < 2; ++cc) {
+            float o[32];
+            const uint32_t ta = tO + lane_base + hh * 64 + cc * 32;
+            tmem_ld32(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(ta, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (!fail) {
+        tc_fence_after();
+        // column c of P buffer b holds the f16 pair (key 2c, 2c+1); this half
+        // writes columns 32 hh .. 32 hh + 31
+        tmem_st32(tP + lane_base + b * (BN / 2) + hh * 32, reinterpret_cast<const float*>(pk));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&B->p_full[b]);
+      }
+    }
+    // epilogue: O / l after the last O += P V; every softmax thread reaches
+    // this barrier once, whether the loop ended or was left together
+    if (!fail)
+      fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[(nkt - 1) & 1],
+                                                    ((nkt - 1) >> 1) & 1, B, p.dev_err));
+    red_sum[hh * BM + r] = l;
+    if (!named_bar_or(2, LY::kSoftWarps * 32, fail)) {
+      tc_fence_after();
+      const float lt = l + red_sum[(hh ^ 1) * BM + r];
+      const float inv = (lt > 0.f) ? p.out_mul / lt : 0.f;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                           ((size_t)(q0 + (row_valid ? i : 0)) * p.n_q + (size_t)kvh * G + g) * D +
+                           hh * 64;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float o[32];
+        tmem_ld32(tO + lane_base + hh * 64 + cc * 32, o);
+        tmem_wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack2<true>(o[e] * inv, o[e + 1] * inv);
+            v.y = pack2<true>(o[e + 2] * inv, o[e + 3] * inv);
+            v.z = pack2<true>(o[e + 4] * inv, o[e + 5] * inv);
+            v.w = pack2<true>(o[e + 6] * inv, o[e + 7] * inv);
+            *reinterpret_cast<uint4*>(out + cc * 32 + e) = v;
+          }
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax

@@ -5,8 +5,14 @@ full-size mixed-step prefill (2 chunks x 512 queries over a 4096-token paged
 history, fp8 cache) is compared on sampled (query, head) rows, each of which
 the oracle computes as attention over that query's causal prefix.  Every case
 runs both ways the call can go: each query tile widening the K/V it reads,
-and with a workspace (the history widened once per chunk and kv head); the two
-feed the tensor cores the same f16 operands and must agree bit for bit.
+and with a workspace (the history widened once per chunk and kv head).  The two
+feed the tensor cores the same f16 K and V.  The workspace kernel splits each
+row's softmax over two warps (half a tile each): it decides per half whether
+masking is needed, so an exponent argument may come from one fused
+multiply-add instead of a multiply and an add (flipping the f16 rounding of
+that P now and then), and it adds the row sum as two partial sums.  The two
+paths therefore agree to a bound far inside the oracle tolerance, not bit
+for bit.
 """
 import numpy as np
 import pytest
@@ -38,6 +44,15 @@ def _run(B, inp, dev, max_chunk_len, staged=False):
                        max_chunk_len, inp.k_scale, inp.v_scale, workspace=ws, dev_err=err)
     torch.cuda.synchronize()
     return out.float().cpu().numpy().astype(np.float64), int(err.item())
+
+
+def _paths_agree(a, b):
+    """The two paths' outputs (bf16 values as float64): within one bf16 ulp
+    plus 2^-12 (a P that rounds to the neighbouring f16 moves an output by
+    far less), and mostly identical."""
+    assert np.isfinite(a).all() and np.isfinite(b).all()
+    assert (np.abs(a - b) <= np.abs(a) * 2.0 ** -7 + 2.0 ** -12).all()
+    assert np.mean(a == b) > 0.5
 
 
 def _oracle(inp):
@@ -85,7 +100,7 @@ def test_chunk_lengths_at_tile_edges(B, cuda_device, staged):
 
 
 @pytest.mark.parametrize("kv_dt", [W.FP8_E4M3, W.BF16])
-def test_workspace_and_in_kernel_widening_agree_bit_for_bit(B, cuda_device, kv_dt):
+def test_workspace_and_in_kernel_widening_agree(B, cuda_device, kv_dt):
     # contexts ending inside a block, on a 128-key tile edge and one past it
     spec = W.PrefillSpec("agree", 4, 0, 0, 16, 4, 128, W.BF16, kv_dt, extra_blocks=3, seed=313)
     chunk_lens = [100, 7, 128, 1]
@@ -94,7 +109,7 @@ def test_workspace_and_in_kernel_widening_agree_bit_for_bit(B, cuda_device, kv_d
     a, ea = _run(B, inp, cuda_device, 128, staged=False)
     b, eb = _run(B, inp, cuda_device, 128, staged=True)
     assert ea == eb == 0
-    assert np.array_equal(a, b)
+    _paths_agree(a, b)
 
 
 def test_out_of_range_block_id_is_flagged_on_both_paths(B, cuda_device):
@@ -107,7 +122,8 @@ def test_out_of_range_block_id_is_flagged_on_both_paths(B, cuda_device):
     a, ea = _run(B, inp, cuda_device, 40, staged=False)
     b, eb = _run(B, inp, cuda_device, 40, staged=True)
     assert ea & 1 and eb & 1  # PA_DEVERR_BLOCK_ID
-    assert np.isfinite(b).all() and np.array_equal(a, b)
+    assert np.isfinite(b).all()
+    _paths_agree(a, b)
 
 
 @pytest.mark.parametrize("staged", [False, True])
