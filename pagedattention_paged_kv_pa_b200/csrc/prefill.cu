@@ -611,15 +611,19 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         tmem_ld32(tSrow + 32, x + 32);
         tmem_wait_ld();
         if (full) {
+          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
-          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, x[e]);
+          for (int e = 0; e < 64; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[e]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           mx *= sl;
         } else {
+          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int e = 0; e < 64; ++e) {
             const bool vis = !row_valid || (kbase + e <= lim);
-            mx = fmaxf(mx, vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
+            m4[e & 3] = fmaxf(m4[e & 3], vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
           }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
       }
       red_max[((j & 1) * 2 + hh) * BM + r] = mx;
@@ -639,7 +643,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         m_used = m_new;
       }
       // pass 2: P = 2^(s*scale - m) as f16 pairs
-      float rs = 0.f;
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum in 4 chains
       uint32_t pk[32];
       const float neg_m = -m_used;
       {
@@ -652,7 +656,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           for (int e = 0; e < 64; e += 2) {
             const float a = fast_exp2(fmaf(x[e], sl, neg_m));
             const float bb = fast_exp2(fmaf(x[e + 1], sl, neg_m));
-            rs += a + bb;
+            r4[(e >> 1) & 3] += a + bb;
             pk[e / 2] = pack2<false>(a, bb);
           }
         } else {
@@ -662,14 +666,14 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             const float v0 = row_valid ? (k0 <= lim ? x[e] * sl : -INFINITY) : 0.f;
             const float v1 = row_valid ? (k0 + 1 <= lim ? x[e + 1] * sl : -INFINITY) : 0.f;
             const float a = fast_exp2(v0 + neg_m), bb = fast_exp2(v1 + neg_m);
-            rs += a + bb;
+            r4[(e >> 1) & 3] += a + bb;
             pk[e / 2] = pack2<false>(a, bb);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&B->s_empty[s]);  // S buffer s may be overwritten by S(j+2)
-      l += rs;
+      l += (r4[0] + r4[1]) + (r4[2] + r4[3]);
       const int b = j & 1;
       // P buffer b is free once O += P V of tile j-2 has completed
       if (j >= 2)
@@ -765,8 +769,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           tmem_ld32(tSrow + cc * 32, x);
           tmem_ld32(tSrow + cc * 32 + 32, x + 32);
           tmem_wait_ld();
+          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
-          for (int e = 0; e < 64; ++e) mx = fmaxf(mx, x[e]);
+          for (int e = 0; e < 64; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[e]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
         mx *= sl;
       } else {
@@ -775,11 +781,13 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           float x[32];
           tmem_ld32(tSrow + cc * 32, x);
           tmem_wait_ld();
+          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const bool vis = !row_valid || (kbase + cc * 32 + e <= lim);
-            mx = fmaxf(mx, vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
+            m4[e & 3] = fmaxf(m4[e & 3], vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
           }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
       }
       // O and l are rescaled lazily: only when the max grew by more than 2^8
@@ -793,7 +801,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       }
       // pass 2: P = 2^(s*scale - m) as f16, kept in registers until the P
       // buffer is free
-      float rs = 0.f;
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum in 4 chains
       uint32_t pk[BN / 2];
       const float neg_m = -m_used;
       if (full) {
@@ -806,7 +814,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           for (int e = 0; e < 32; e += 2) {
             const float a = fast_exp2(fmaf(x[e], sl, neg_m));
             const float bb = fast_exp2(fmaf(x[e + 1], sl, neg_m));
-            rs += a + bb;
+            r4[(e >> 1) & 3] += a + bb;
             pk[cc * 16 + e / 2] = pack2<false>(a, bb);
           }
         }
@@ -822,14 +830,14 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             const float v0 = row_valid ? (k0 <= lim ? x[e] * sl : -INFINITY) : 0.f;
             const float v1 = row_valid ? (k0 + 1 <= lim ? x[e + 1] * sl : -INFINITY) : 0.f;
             const float a = fast_exp2(v0 + neg_m), bb = fast_exp2(v1 + neg_m);
-            rs += a + bb;
+            r4[(e >> 1) & 3] += a + bb;
             pk[cc * 16 + e / 2] = pack2<false>(a, bb);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&B->s_empty[s]);  // S buffer s may be overwritten by S(j+2)
-      l += rs;
+      l += (r4[0] + r4[1]) + (r4[2] + r4[3]);
       const int b = j & 1;
       // P buffer b is free once O += P V of tile j-2 has completed
       if (j >= 2) {
