@@ -8,35 +8,47 @@
 // they run on the 5th-generation tensor cores with accumulators in TMEM.
 //
 // CTA tile: M = 128 rows = (128 / G) consecutive queries x the G query heads
-// of one kv head (GQA packing: each K/V tile is widened once for the whole
-// group).  Keys are processed in tiles of 128 (8 blocks of 16 from the block
-// table).  Warp roles (288 threads):
-//   warps 0-3  softmax: thread r owns row r = TMEM lane r; reads S from TMEM,
-//              masks, keeps an online max/sum, writes P (f16) back to TMEM,
-//              rescales the TMEM output only when its max grew by more than
-//              2^8, and writes the normalised output at the end;
-//   warps 4-7  K/V converters: load a tile's K and V rows through the block
-//              table with coalesced 16-byte loads, widen fp8 codes exactly to
-//              f16 (K on the conversion pipe; V on the integer pipe as
-//              code x 2^-8, folded into the output scale; bf16 values are
-//              converted to f16) and write both as [key][d] rows in the
-//              128-byte-swizzled layout: K-major for K, MN-major for V, so V
-//              needs no transpose;
+// of one kv head (GQA packing: each K/V tile serves the whole group).  Keys
+// are processed in tiles of 128 (8 blocks of 16 from the block table).  The
+// products run in f16, so K and V are widened first, in one of two ways:
+//
+// With a workspace (kStaged, 320 threads): prefill_widen_kernel first writes
+// each chunk's history, per kv head, as f16 rows (zeros past the context), so
+// the 16 query tiles of a 512-query chunk share one widening instead of each
+// doing its own.  Then:
+//   warps 0-7  softmax, two warps per row: warps w and w+4 own rows
+//              32 (w%4) .. +31 (TMEM lanes) and take half a key tile each;
+//              they read S from TMEM, mask, keep an online max/sum (the
+//              halves' maxima meet in shared memory at a named barrier),
+//              write P (f16) back to TMEM, rescale their half of the TMEM
+//              output only when the max grew by more than 2^8, and write the
+//              normalised output at the end;
 //   warp 8     TMEM owner and MMA issuer (one elected lane): S = Q K^T into a
 //              double-buffered TMEM score tile, O += P V into TMEM with P
-//              read from TMEM (the softmax writes P there, double-buffered).
-// K tiles (2 stages) are released as soon as S = Q K^T has read them, V tiles
-// (4 stages) once O += P V has, so the converters run up to four tiles ahead
-// of the P V products.
+//              read from TMEM (double-buffered);
+//   warp 9     TMA producer: two 64-column boxes per operand straight from
+//              the workspace into 3 K and 2 V stages (128-byte swizzle).
+//
+// Without one (kWidenFp8 320 threads, kWidenBf16 288): one softmax warp per
+// row (warps 0-3), the MMA warp 8, and converter warps 4-7 that widen each
+// tile themselves and write both operands as [key][d] rows in the
+// 128-byte-swizzled layout (K-major for K, MN-major for V, so V needs no
+// transpose): fp8 codes exactly to f16 (K on the conversion pipe; V on the
+// integer pipe as code x 2^-8, folded into the output scale), bf16 values
+// converted to f16.  With an fp8 cache warp 9 brings each tile's raw rows
+// into a 2-stage shared-memory ring by TMA, two tiles ahead.
+//
 // Both MMAs run in f16 with fp32 accumulation: every E4M3 value is exact in
 // f16, bf16 inputs are exact while inside f16's range (|x| <= 65504; below
 // 2^-14 they keep an absolute precision of 2^-24), and P gets 11 significant
-// bits instead of bf16's 8.
-// S(j+1) is issued before O += P(j) V(j), so the next tile's QK^T overlaps
-// this tile's softmax.  All waits are
-// bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA drains its
-// tensor-core work and frees its TMEM before returning.
+// bits instead of bf16's 8.  K stages are released as soon as S = Q K^T has
+// read them, V stages once O += P V has.  S(j+1) is issued before
+// O += P(j) V(j), so the next tile's QK^T overlaps this tile's softmax.  All
+// waits are bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA
+// drains its tensor-core work and loads in flight and frees its TMEM before
+// returning.
 #include <type_traits>
+#include <utility>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -252,7 +264,9 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
   Bars* B = reinterpret_cast<Bars*>(smem + kBarOff);
   const uint32_t sbase = smem_u32(smem);
 
-  const int tile = blockIdx.x, kvh = blockIdx.y, c = blockIdx.z;
+  // query tiles later in a chunk see more keys (causal): they are launched
+  // first, so the shorter ones fill the last wave
+  const int tile = gridDim.x - 1 - blockIdx.x, kvh = blockIdx.y, c = blockIdx.z;
   const int G = p.group;
   const int QT = BM / G;  // queries per CTA tile
   const int q0 = p.query_start_loc[c], q1 = p.query_start_loc[c + 1];
@@ -378,6 +392,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       if (lane == 0) {
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
+        // launched as a programmatic dependent of the widening pass: the
+        // prologue above overlapped it; the workspace is read only after it
+        // has completed
+        pdl_wait();
         const int row0 = (c * p.n_kv + kvh) * p.stage_rows;
         int issued_k = 0, issued_v = 0;
         for (int j = 0; j < nkt; ++j) {
@@ -923,6 +941,10 @@ __global__ void __launch_bounds__(256)
                          const void* __restrict__ v_pool, uint16_t* __restrict__ kst,
                          uint16_t* __restrict__ vst) {
   const int t = blockIdx.x, kvh = blockIdx.y, c = blockIdx.z;
+  // launched as a programmatic dependent: whatever ran before (the slot
+  // write) completes first; then the attention kernel may start its prologue
+  pdl_wait();
+  pdl_launch_dependents();
   const int ctx = p.context_lens[c];
   if (ctx < 0 || ctx > p.max_blocks * 16) return;  // the attention kernel flags it
   const int k0 = t * BN;
@@ -971,6 +993,25 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// a launch that may begin before the previous kernel in the stream has
+// finished (programmatic dependent launch; the kernel calls pdl_wait before
+// it reads what that kernel wrote)
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int MODE>
 cudaError_t launch_tc(const PrefillParams& p, const void* k_pool, const void* v_pool,
                       const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t st) {
@@ -980,6 +1021,9 @@ cudaError_t launch_tc(const PrefillParams& p, const void* k_pool, const void* v_
   if (attr != cudaSuccess) return attr;
   const int QT = BM / p.group;
   dim3 grid((p.max_chunk_len + QT - 1) / QT, p.n_kv, p.n_chunks);
+  if constexpr (MODE == kStaged)  // right after the widening pass
+    return launch_dependent(prefill_tc_kernel<MODE>, grid, dim3(LY::kThreads), LY::kSmemBytes,
+                            st, p, k_pool, v_pool, *tmk, *tmv);
   prefill_tc_kernel<MODE>
       <<<grid, LY::kThreads, LY::kSmemBytes, st>>>(p, k_pool, v_pool, *tmk, *tmv);
   return cudaGetLastError();
@@ -998,11 +1042,11 @@ cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k
   uint16_t* kst = static_cast<uint16_t*>(workspace);
   uint16_t* vst = kst + (size_t)p.n_chunks * p.n_kv * p.stage_rows * D;
   const dim3 grid(p.stage_rows / BN, p.n_kv, p.n_chunks);
-  if (fp8)
-    prefill_widen_kernel<true><<<grid, 256, 0, st>>>(p, k_pool, v_pool, kst, vst);
-  else
-    prefill_widen_kernel<false><<<grid, 256, 0, st>>>(p, k_pool, v_pool, kst, vst);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e =
+      fp8 ? launch_dependent(prefill_widen_kernel<true>, grid, dim3(256), 0, st, p, k_pool,
+                             v_pool, kst, vst)
+          : launch_dependent(prefill_widen_kernel<false>, grid, dim3(256), 0, st, p, k_pool,
+                             v_pool, kst, vst);
   if (e != cudaSuccess) return e;
   return launch_tc<kStaged>(p, k_pool, v_pool, tmk, tmv, st);
 }
