@@ -557,7 +557,7 @@ def run_mixed(args, rank, world, local):
         "prefill_alone": {"us": round(pre_ms * 1e3, 2), "algorithmic_flop": int(flops),
                           "achieved_tflops": round(pre_tflops, 1),
                           "peak_tflops": tflops_peak, "frac": round(pre_tflops / tflops_peak, 4),
-                          "peak_source": tsrc, "includes": "slot write + prefill kernel"},
+                          "peak_source": tsrc, "includes": "slot write + widening pass + prefill kernel"},
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(dec_gbs / peak, 4),
                      "traffic": traffic_from_profile("mixed_step_fp8_decode"),
