@@ -156,6 +156,7 @@ def describe(spec, ctx, num_blocks):
 def get_spec(name):
     from pagedattention_paged_kv_pa_b200 import workloads as W
     return {"llama3_70b_gqa_bf16": W.LLAMA3_70B_GQA_BF16, "llama2_7b_fp16": W.LLAMA2_7B_FP16,
+            "llama3_70b_gqa_bf16_ctx8k": W.LLAMA3_70B_GQA_BF16_CTX8K,
             "mixed_step_fp8_decode": W.MIXED_DECODE_FP8, "tiny_fp32": W.TINY_FP32}[name]
 
 

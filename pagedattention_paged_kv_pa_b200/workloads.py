@@ -182,12 +182,15 @@ LLAMA2_7B_FP16 = DecodeSpec("llama2_7b_fp16", 64, 32, 32, 128, F16, F16, "unifor
 LLAMA3_70B_GQA_BF16 = DecodeSpec("llama3_70b_gqa_bf16", 128, 64, 8, 128, BF16, BF16,
                                  "lognormal", (2048.0, 0.5, 16, 8192), max_ctx=8192,
                                  seed=1003)
+# the same layer with every context at its 8192-token maximum (4.3 GB of K/V)
+LLAMA3_70B_GQA_BF16_CTX8K = DecodeSpec("llama3_70b_gqa_bf16_ctx8k", 128, 64, 8, 128, BF16, BF16,
+                                       "fixed", ((8192,) * 128,), max_ctx=8192, seed=1003)
 # decode half of the mixed continuous-batching step (fp8 KV, per-tensor scale)
 MIXED_DECODE_FP8 = DecodeSpec("mixed_step_fp8_decode", 256, 32, 8, 128, BF16, FP8_E4M3,
                               "uniform", (64, 8192), max_ctx=8192, seed=1005)
 
 SPECS = {s.name: s for s in (TINY_FP32, LLAMA2_7B_FP16, LLAMA3_70B_GQA_BF16,
-                             MIXED_DECODE_FP8)}
+                             LLAMA3_70B_GQA_BF16_CTX8K, MIXED_DECODE_FP8)}
 
 # Draft-token verification ("LLM inference optimization", §五: the target model
 # checks K = 5 draft tokens in one forward pass): the Llama-3-70B GQA layer's

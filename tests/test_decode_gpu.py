@@ -128,7 +128,8 @@ def test_out_of_range_block_id_is_flagged_not_read(B, cuda_device):
     assert np.isfinite(gpu[1]).all()
 
 
-@pytest.mark.parametrize("spec", [W.LLAMA2_7B_FP16, W.LLAMA3_70B_GQA_BF16, W.MIXED_DECODE_FP8],
+@pytest.mark.parametrize("spec", [W.LLAMA2_7B_FP16, W.LLAMA3_70B_GQA_BF16,
+                                  W.LLAMA3_70B_GQA_BF16_CTX8K, W.MIXED_DECODE_FP8],
                          ids=lambda s: s.name)
 def test_full_size_sampled(B, cuda_device, spec):
     """Full-size workload in the benchmark's launch configuration; the oracle
