@@ -99,6 +99,28 @@ def test_chunk_lengths_at_tile_edges(B, cuda_device, staged):
     P.assert_close(gpu, _oracle(inp), W.BF16, W.FP8_E4M3, "prefill tile edges")
 
 
+@pytest.mark.parametrize("staged", [False, True])
+def test_empty_chunks_between_others(B, cuda_device, staged):
+    # a chunk with no queries (its history is still widened, nothing is
+    # written), and an empty sequence (no history, no queries) at the end
+    spec = W.PrefillSpec("empty", 4, 0, 0, 32, 8, 128, W.BF16, W.FP8_E4M3, seed=315)
+    inp = W.make_prefill_inputs(spec, chunk_lens=[20, 0, 33, 0], histories=[100, 50, 0, 0])
+    gpu, err = _run(B, inp, cuda_device, 33, staged)
+    assert err == 0
+    P.assert_close(gpu, _oracle(inp), W.BF16, W.FP8_E4M3, "prefill with empty chunks")
+
+
+@pytest.mark.parametrize("staged", [False, True])
+def test_long_chunk_many_query_tiles(B, cuda_device, staged):
+    # 700 queries = 21 full query tiles of 32 (G = 4) and a ragged one, over
+    # 1,033 keys (8 full key tiles and a ragged one)
+    spec = W.PrefillSpec("long", 1, 0, 0, 32, 8, 128, W.BF16, W.BF16, seed=316)
+    inp = W.make_prefill_inputs(spec, chunk_lens=[700], histories=[333])
+    gpu, err = _run(B, inp, cuda_device, 700, staged)
+    assert err == 0
+    P.assert_close(gpu, _oracle(inp), W.BF16, W.BF16, "prefill, one long chunk")
+
+
 @pytest.mark.parametrize("kv_dt", [W.FP8_E4M3, W.BF16])
 def test_workspace_and_in_kernel_widening_agree(B, cuda_device, kv_dt):
     # contexts ending inside a block, on a 128-key tile edge and one past it
