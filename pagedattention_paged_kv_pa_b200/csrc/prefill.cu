@@ -60,7 +60,6 @@ namespace {
 constexpr int D = 128;       // head dim
 constexpr int BM = 128;      // rows per CTA tile
 constexpr int BN = 128;      // keys per tile
-constexpr int kSoftmaxWarps = 4;
 // TMEM columns: S[2] (2 x 128 fp32), O (128 fp32), P[2] (2 x 64 columns of f16 pairs)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
@@ -468,7 +467,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
   } else if (warp >= LY::kSoftWarps) {
     // ------------------------------------------------------------ converters
     if constexpr (!LY::kStagedOps) {
-    const int ct = tid - kSoftmaxWarps * 32;  // 0..127
+    const int ct = tid - LY::kSoftWarps * 32;  // 0..127
     const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
     const int kv_es = FP8 ? 1 : 2;
     // block ids of a tile's 8 blocks (-1 past the context); the next tile's
