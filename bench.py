@@ -563,7 +563,8 @@ def run_mixed(args, rank, world, local):
                      "frac": round(dec_gbs / peak, 4),
                      "traffic": traffic_from_profile("mixed_step_fp8_decode"),
                      "kernel": "decode_mma_kernel (fp8 cache)"},
-        "gpu_launches": 5 * K,
+        # per step: two slot writes, decode partition + merge, widening pass + prefill
+        "gpu_launches": 6 * K,
         "clocks": clocks,
     }
     if rank == 0:
