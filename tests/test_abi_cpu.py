@@ -211,3 +211,8 @@ def test_prefill_workspace_size_and_refusals(B):
     assert _pre(B, nq=6, nkv=4) == B.PA_ERR_INVALID_ARG
     assert _pre(B, nb=1 << 27, nkv=2) == B.PA_ERR_UNSUPPORTED        # pool rows >= 2^31
     assert _pre(B, nc=0) == B.PA_OK                                   # nothing to do
+    # workspace rows (chunks x kv heads x max_blocks*16 rounded up to 128) >= 2^31
+    big = dict(nc=65535, nq=16, nkv=16, mb=2048)
+    need_big = B.pa_prefill_workspace_size(65535, 16, 128, 2048)
+    assert need_big == 2 * 65535 * 16 * 32768 * 128 * 2
+    assert _pre(B, ws=4096, wsb=need_big, **big) == B.PA_ERR_UNSUPPORTED
