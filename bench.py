@@ -164,8 +164,9 @@ def get_spec(name):
 # CPU oracle timing (baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(inp, budget_s: float, max_units=None):
-    """Time the oracle on a bounded prefix of the workload's sequences.
+def oracle_sample(inp, budget_s: float, max_units=None, threads=None):
+    """Time the oracle on a bounded prefix of the workload's sequences, on
+    `threads` host threads (default: all cores).
     Returns (seconds, bytes, seqs, tokens, threads)."""
     import oracle as orc
     from pagedattention_paged_kv_pa_b200 import workloads as W
@@ -174,7 +175,7 @@ def oracle_sample(inp, budget_s: float, max_units=None):
     bt = inp.block_tables.cpu().numpy()
     cl = inp.context_lens.cpu().numpy()
     kp, vp = inp.k_pool, inp.v_pool
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     done_s, done_bytes, done_seqs, done_tok = 0.0, 0, 0, 0
     s = 0
     chunk = max(1, threads // max(1, spec.n_kv_heads) or 1)
@@ -401,6 +402,12 @@ def run_ours(args, rank, world, local):
                                 "kind": "oracle",
                                 "sample": f"first {ns} of {n} sequences ({nt} tokens) of the "
                                           f"same workload, {secs:.1f} s, fp64 C oracle"}
+        # the same oracle on one host thread (a smaller sample)
+        secs1, b1, ns1, nt1, _ = oracle_sample(inp, budget_s=min(3.0, args.cpu_budget),
+                                               threads=1)
+        line["cpu_baseline"]["single_thread"] = {
+            "value": round(b1 / secs1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "sample": f"first {ns1} sequences ({nt1} tokens), {secs1:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
