@@ -104,6 +104,10 @@ const char* pa_status_string(pa_status s);
  * Supported: block_size 16; head_dim 64 or 128; n_q_heads % n_kv_heads == 0
  * with group size n_q_heads / n_kv_heads <= 8; (q_dtype, kv_dtype) in
  * {(F32,F32), (F16,F16), (BF16,BF16), (F16,FP8_E4M3), (BF16,FP8_E4M3)}.
+ * 16-bit caches multiply in the cache's type; with an fp8 cache the E4M3
+ * values widen to f16 exactly and a bf16 query head is multiplied by a power
+ * of two that puts its largest magnitude in [2^14, 2^15) before its f16
+ * rounding, its scores by the inverse, so the whole bf16 range is taken.
  * Pointers must be 16-byte aligned.  Output rows are bit-identical under any
  * permutation of the physical blocks (partitioning and reduction order depend
  * only on logical positions).
@@ -154,9 +158,13 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
  *     out[s][i][h] = softmax(scale * q[s][i][h] . K_s[0..c_i]^T) . V_s[0..c_i]
  * A query whose position is negative (context_lens[s] < q_len - i) has no
  * keys and gets an all-zero row.  This is the causal chunk of
- * pa_prefill_paged with history context_lens[s] - q_len, computed the way
- * decode is: each K/V tile is read once for all of a sequence's queries of a
- * kv head (up to 8 (query, head) pairs per tile pass), HBM-bound.
+ * pa_prefill_paged with history context_lens[s] - q_len, and each K/V tile is
+ * read once for all of a sequence's queries of a kv head: with bf16 queries,
+ * head_dim 128, a bf16 or fp8 cache and group size 1, 2, 4 or 8 it runs on
+ * pa_prefill_paged's tensor-core kernel (one 128-row tile holds the q_len x G
+ * (query, head) rows of a kv head; no partitions, so the workspace is not
+ * written), otherwise on decode's partition and merge kernels with up to 32
+ * (query, head) pairs per tile pass.
  *
  *   out, q       device [num_seqs][q_len][n_q_heads][head_dim], dtype q_dtype
  *   q_len        1 .. 8 (1 gives pa_decode's result)
@@ -248,9 +256,13 @@ pa_status pa_prefix_groups(const int32_t* block_tables, const int32_t* context_l
  *  - Returns PA_ERR_UNSUPPORTED before any launch when the call would need more
  *    scratch than that, i.e. when pa_decode_workspace_size(num_seqs, n_q_heads,
  *    head_dim, max_blocks_per_seq) > pa_decode_noalloc_scratch_bytes().
- *  - The first call on a device looks up the array's device address with that
- *    device current and caches it; make that first call before any stream
- *    capture.
+ *  - The array's device address belongs to a CUDA context.  The first call
+ *    made with a given context current (the device's primary context, or a
+ *    driver-API context the caller made current) looks it up and caches it
+ *    under that context's id; make that first call before any stream capture.
+ *    A context created later (for instance after cudaDeviceReset) has a new
+ *    id and gets a fresh lookup, so an address cached for a destroyed context
+ *    is never used.
  *  - All calls share the one array, which keeps the last call's contents:
  *    calls whose work overlaps on the GPU (other streams, other host threads)
  *    race on it and must be ordered by the caller.  Nothing in it needs to
@@ -289,24 +301,33 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_pool, const 
  *   max_chunk_len  host bound on every L_c (sizes the grid; no device sync)
  *
  * Supported: block_size 16, head_dim 128, group size 1, 2, 4 or 8, q_dtype
- * BF16 and kv_dtype BF16 or FP8_E4M3.  The products run in f16 with fp32
- * accumulation: E4M3 values widen to f16 exactly; bf16 q/K/V values are exact
- * in f16 while |x| <= 65504 (values below 2^-14 keep an absolute precision of
- * 2^-24; larger magnitudes overflow), a restriction the bf16-cache variant
- * carries.  A block id outside [0, num_blocks) is flagged with
- * PA_DEVERR_BLOCK_ID and its keys read as zeros.  The output is written in
- * q_dtype.  PA_ERR_UNSUPPORTED also when num_blocks * n_kv_heads * 16 >= 2^31
- * (the pools are addressed as that many rows of head_dim elements).
+ * BF16 and kv_dtype BF16 or FP8_E4M3.  Both products accumulate in fp32 and
+ * take every input value exactly, over the whole bf16 range ([P2] "兩層實作":
+ * paging leaves the math unchanged):
+ *  - bf16 cache: q, K and V enter the tensor cores as bf16; the softmax
+ *    weights P enter O += P V as a bf16 value plus its bf16 rounding residual
+ *    (about 16 significant bits);
+ *  - fp8 cache: E4M3 values widen to f16 exactly; each bf16 query row is
+ *    multiplied by a power of two that puts its largest magnitude in
+ *    [2^14, 2^15) before its f16 rounding and its scores by the inverse (an
+ *    element below 2^-28 of its row's largest keeps an absolute precision of
+ *    2^-39 of that largest); P is f16.
+ * A block id outside [0, num_blocks) is flagged with PA_DEVERR_BLOCK_ID and
+ * its keys read as zeros.  The output is written in q_dtype.
+ * PA_ERR_UNSUPPORTED also when num_blocks * n_kv_heads * 16 >= 2^31 (the pools
+ * are addressed as that many rows of head_dim elements).
  *
  *   workspace      NULL, or device memory of at least
  *                  pa_prefill_workspace_size(n_chunks, n_kv_heads, head_dim,
  *                  max_blocks_per_seq, block_size) bytes, 16-byte aligned,
  *                  owned by the caller and free for this call's duration.
- * With NULL every query tile widens the K/V it reads to f16 itself.  With a
- * workspace a first kernel widens each chunk's history once (per kv head)
- * into it, and the tensor-core kernel streams the f16 operands from there;
- * every query tile of a chunk shares them.  The results are identical up to
- * the order of the fp32 accumulation (the same f16 operands either way).
+ * fp8 cache: with NULL every query tile widens the K/V it reads to f16
+ * itself; with a workspace a first kernel widens each chunk's history once
+ * (per kv head) into it, and the tensor-core kernel streams the f16 operands
+ * from there, every query tile of a chunk sharing them.  The results are
+ * identical up to the order of the fp32 accumulation (the same f16 operands
+ * either way).  bf16 cache: the kernel reads the pool's blocks directly and
+ * a workspace, if given, is checked but not used.
  * PA_ERR_INVALID_ARG if the workspace is too small or misaligned;
  * PA_ERR_UNSUPPORTED if n_chunks * n_kv_heads * (max_blocks_per_seq * 16
  * rounded up to 128) >= 2^31.

@@ -174,6 +174,18 @@ size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim, int m
   return ws_total_bytes(s);
 }
 
+// pa_decode_multi's step is the causal chunk of a sequence's q_len newest
+// queries over its cache, so for bf16 queries over a bf16 or fp8 cache with
+// head_dim 128 and group 1, 2, 4 or 8 it runs on the chunked-prefill
+// tensor-core kernel: one 128-row tile per (sequence, kv head) holds all
+// q_len x G (query, head) rows and reads each K/V tile once for them.
+static bool multi_on_tensor_cores(int q_len, int head_dim, int group, pa_dtype q_dt,
+                                  pa_dtype kv_dt) {
+  return q_len > 1 && head_dim == 128 && q_dt == PA_BF16 &&
+         (kv_dt == PA_BF16 || kv_dt == PA_FP8_E4M3) &&
+         (group == 1 || group == 2 || group == 4 || group == 8);
+}
+
 static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool, const void* v_pool,
                                const int32_t* block_tables, const int32_t* context_lens,
                                float scale, int block_size, int n_q_heads, int n_kv_heads,
@@ -184,7 +196,7 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
                                const int32_t* grp_members = nullptr,
                                const int32_t* grp_shared_blocks = nullptr,
                                const int32_t* seq_group = nullptr, int n_groups = 0,
-                               int grp_width = 0) {
+                               int grp_width = 0, bool tensor_core_multi = false) {
   DecodeShape s{n_q_heads, n_kv_heads, head_dim, num_seqs, max_blocks_per_seq, num_blocks,
                 pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   pa_status st = check_decode(s, block_size, q_dtype, kv_dtype);
@@ -246,6 +258,27 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
       return PA_ERR_CUDA;
   }
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (tensor_core_multi) {
+    pa::PrefillParams pp;
+    pp.out = out;
+    pp.q = q;
+    pp.block_tables = block_tables;
+    pp.query_start_loc = nullptr;
+    pp.context_lens = context_lens;
+    pp.dev_err = dev_err;
+    pp.scale_log2 = p.scale_log2;
+    pp.out_mul = p.out_mul;  // the in-kernel widening takes fp8 V as code x 2^-8 too
+    pp.n_q = n_q_heads;
+    pp.n_kv = n_kv_heads;
+    pp.group = p.group;
+    pp.n_chunks = num_seqs;
+    pp.max_blocks = max_blocks_per_seq;
+    pp.num_blocks = num_blocks;
+    pp.max_chunk_len = q_len;
+    pp.stage_rows = static_cast<int>(pa::prefill_stage_rows(max_blocks_per_seq));
+    pp.fixed_q_len = q_len;
+    return cuda_status(pa::launch_prefill(pp, kv_dtype, k_pool, v_pool, &tmk, &tmv, nullptr, cs));
+  }
   if (n_groups > 0) {
     // one launch: the groups' shared partitions, every member at once (one
     // column per (member, head)), next to every sequence's other partitions
@@ -333,11 +366,15 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_pool, const vo
                           pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
                           void* workspace, size_t workspace_bytes, int32_t* dev_err,
                           void* stream) {
+  const bool tc = n_kv_heads > 0 && n_q_heads % n_kv_heads == 0 &&
+                  multi_on_tensor_cores(q_len, head_dim, n_q_heads / n_kv_heads, q_dtype,
+                                        kv_dtype);
   pa_status st = decode_parts_impl(out, q, k_pool, v_pool, block_tables, context_lens, scale,
                                    block_size, n_q_heads, n_kv_heads, head_dim, num_seqs, q_len,
                                    max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
-                                   v_scale, workspace, workspace_bytes, dev_err, stream);
-  if (st != PA_OK) return st;
+                                   v_scale, workspace, workspace_bytes, dev_err, stream, nullptr,
+                                   nullptr, nullptr, 0, 0, tc);
+  if (st != PA_OK || tc) return st;  // the tensor-core route has no partitions to merge
   return decode_reduce_impl(out, context_lens, n_q_heads * q_len, head_dim, num_seqs,
                             max_blocks_per_seq, q_dtype, kv_dtype, v_scale, workspace,
                             workspace_bytes, stream);
@@ -493,7 +530,8 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
   p.context_lens = context_lens;
   p.dev_err = dev_err;
   p.scale_log2 = scale * kLog2e * (fp8 ? k_scale : 1.f);
-  p.out_mul = fp8 ? v_scale * kFp8VUnscale : 1.f;  // fp8 V is widened as code x 2^-8
+  // in-kernel widening takes fp8 V as code x 2^-8 (see below for the workspace)
+  p.out_mul = fp8 ? v_scale * kFp8VUnscale : 1.f;
   p.n_q = n_q_heads;
   p.n_kv = n_kv_heads;
   p.group = G;
@@ -502,14 +540,23 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
   p.num_blocks = num_blocks;
   p.max_chunk_len = max_chunk_len;
   p.stage_rows = static_cast<int>(pa::prefill_stage_rows(max_blocks_per_seq));
+  p.fixed_q_len = 0;
   CUtensorMap tmk{}, tmv{};
-  if (workspace != nullptr) {
+  if (workspace != nullptr &&
+      (!aligned16(workspace) ||
+       workspace_bytes < pa_prefill_workspace_size(n_chunks, n_kv_heads, head_dim,
+                                                   max_blocks_per_seq, block_size)))
+    return PA_ERR_INVALID_ARG;
+  if (!fp8) {
+    // bf16 cache: the tensor cores take the pools' bf16 blocks as they are,
+    // loaded by TMA through the block table; there is nothing to widen, so a
+    // workspace is not used
+    if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
+        !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv))
+      return PA_ERR_CUDA;
+  } else if (workspace != nullptr) {
     // the history of every chunk is widened once into the workspace; both fp8
     // operands widen exactly there, so V needs no 2^-8 fold
-    if (!aligned16(workspace) ||
-        workspace_bytes < pa_prefill_workspace_size(n_chunks, n_kv_heads, head_dim,
-                                                    max_blocks_per_seq, block_size))
-      return PA_ERR_INVALID_ARG;
     const uint64_t rows = (uint64_t)n_chunks * n_kv_heads * p.stage_rows;
     if (rows >= (uint64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
     p.out_mul = fp8 ? v_scale : 1.f;
@@ -517,8 +564,8 @@ pa_status pa_prefill_paged(void* out, const void* q, const void* k_pool, const v
     if (!get_map(kst, rows, 128, 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, &tmk) ||
         !get_map(kst + rows * 128, rows, 128, 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, &tmv))
       return PA_ERR_CUDA;
-  } else if (fp8 && (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
-                     !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv))) {
+  } else if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
+             !kv_pool_map(v_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmv)) {
     return PA_ERR_CUDA;
   }
   return cuda_status(pa::launch_prefill(p, kv_dtype, k_pool, v_pool, &tmk, &tmv, workspace,

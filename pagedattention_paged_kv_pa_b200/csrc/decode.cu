@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
     // 16-dim step so that K can be read as whole 32-bit words; Q uses the
     // same pairing, which leaves the dot products unchanged.
     uint32_t qb[KS][2];
+    float col_scale;  // scale x log2 e (x k_scale) x 2^-e of column g
     {
       bool hv = g < ncols;
       size_t r = 0;
@@ -369,20 +370,40 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
         r = (size_t)seq * p.n_q + (size_t)kvh * G + (hv ? g : 0);
       }
       const QT* qrow = reinterpret_cast<const QT*>(p.q) + r * D;
+      // fp8 cache with bf16 queries: the column's row enters the f16 MMAs
+      // times 2^e (its largest magnitude in [2^14, 2^15)); its scores are
+      // scaled by 2^-e.  The four lanes t of a column hold all of its dims.
+      int e = 0;
+      if constexpr (FP8 && Q_BF16) {
+        uint32_t mag = 0;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const uint2 w = *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * t);
+          mag = max(mag, max(bf16x2_max_mag(w.x), bf16x2_max_mag(w.y)));
+        }
+        mag = hv ? mag : 0u;
+        mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, 1));
+        mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, 2));
+        e = f16_row_shift(mag);
+      }
+      const float up = exp2i(e);
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         if constexpr (FP8) {
           const int d0 = 16 * kk + 4 * t;
-          qb[kk][0] = pack2<false>(to_f32(qrow[d0]), to_f32(qrow[d0 + 1]));
-          qb[kk][1] = pack2<false>(to_f32(qrow[d0 + 2]), to_f32(qrow[d0 + 3]));
+          qb[kk][0] = pack2<false>(to_f32(qrow[d0]) * up, to_f32(qrow[d0 + 1]) * up);
+          qb[kk][1] = pack2<false>(to_f32(qrow[d0 + 2]) * up, to_f32(qrow[d0 + 3]) * up);
         } else {
           qb[kk][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t);
           qb[kk][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 8 + 2 * t);
         }
         if (!hv) qb[kk][0] = qb[kk][1] = 0u;
       }
+      col_scale = p.scale_log2 * exp2i(-e);
     }
-    const float sl = p.scale_log2;
+    // score scales of the lane's two columns 2t, 2t+1 (held by lanes g = 2t, 2t+1)
+    const float sl_a = __shfl_sync(0xffffffffu, col_scale, 8 * t);
+    const float sl_b = __shfl_sync(0xffffffffu, col_scale, 8 * t + 4);
     const uint32_t sbase = smem_u32(smem);
     const int q4 = lane >> 3;
     // multi-query causal limits: keys at positions >= lim are masked for the
@@ -433,7 +454,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(
           }
         }
         // ---- online softmax (log2 domain); lane holds tokens g, g+8 of heads 2t, 2t+1
-        float x0 = sc[0] * sl, x1 = sc[1] * sl, x2 = sc[2] * sl, x3 = sc[3] * sl;
+        float x0 = sc[0] * sl_a, x1 = sc[1] * sl_b, x2 = sc[2] * sl_a, x3 = sc[3] * sl_b;
         if (valid < 16) {
           if (g >= valid) x0 = x1 = -INFINITY;
           if (g + 8 >= valid) x2 = x3 = -INFINITY;

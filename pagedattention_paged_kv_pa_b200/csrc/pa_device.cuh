@@ -216,6 +216,36 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_div256(uint32_t w, uint32_t 
   return (y + (y & 0x00800080u)) << 7;
 }
 
+// Rows of bf16 queries meet f16 operands (fp8 caches widen to f16 exactly):
+// a row is multiplied by 2^e before its f16 rounding, e chosen so that its
+// largest magnitude lands in [2^14, 2^15), and the row's scores by 2^-e after
+// the product.  Both steps are exact (powers of two, no overflow: E4M3 values
+// are below 2^9, so a product stays below 2^24 and a 128-term sum below 2^31);
+// an element keeps all its bits unless it is below 2^-28 of the row's largest,
+// and then its error is at most 2^-39 of that largest -- far under the
+// rounding of the fp32 sum itself.
+
+// The larger magnitude of the two bf16 values in w, as bf16 bits (for values
+// that are not NaN the bits order like the magnitudes).
+__device__ __forceinline__ uint32_t bf16x2_max_mag(uint32_t w) {
+  return max(w & 0x7fffu, (w >> 16) & 0x7fffu);
+}
+// e for a row whose largest magnitude has the bf16 bits `mag` (0 for a zero,
+// infinite or NaN row), clamped to [-110, 110] so that 2^e and a score scale
+// times 2^-e stay normal floats.
+__device__ __forceinline__ int f16_row_shift(uint32_t mag) {
+  if (mag == 0u || mag >= 0x7f80u) return 0;
+  const int ex = mag >= 0x80u ? (int)(mag >> 7) - 127 : -127;  // floor(log2 |x|)
+  return min(max(14 - ex, -110), 110);
+}
+// 2^e as a float, for e in [-126, 127]
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+// two bf16 values times `up` (a power of two), rounded to f16
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float up) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  return pack2<false>(f.x * up, f.y * up);
+}
+
 __device__ __forceinline__ float warp_max_xor(float v, int lo_mask) {
   for (int m = 16; m >= lo_mask; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
   return v;

@@ -110,6 +110,12 @@ struct PrefillParams {
   float out_mul;
   int n_q, n_kv, group, n_chunks, max_blocks, num_blocks, max_chunk_len;
   int stage_rows;  // workspace rows per (chunk, kv head): max_blocks * 16 rounded up to 128
+  // 0: chunk c's queries are query_start_loc[c] .. query_start_loc[c+1]-1.
+  // q_len > 0 (multi-query decode): chunk c is sequence c's q_len queries,
+  // rows c q_len .. c q_len + q_len - 1, at the last q_len positions of its
+  // context; query_start_loc is not read, and queries before the context's
+  // start get all-zero rows.
+  int fixed_q_len;
 };
 // Without a workspace the attention kernel widens K/V itself (tmk / tmv: TMA
 // maps over the fp8 pools, the decode kernel's; unused for bf16).  With one,

@@ -9,44 +9,56 @@
 //
 // CTA tile: M = 128 rows = (128 / G) consecutive queries x the G query heads
 // of one kv head (GQA packing: each K/V tile serves the whole group).  Keys
-// are processed in tiles of 128 (8 blocks of 16 from the block table).  The
-// products run in f16, so K and V are widened first, in one of two ways:
+// are processed in tiles of 128 (8 blocks of 16 from the block table).
+//
+// The paged kernel must not change the math ("vLLM explained", "兩層實作"), so
+// every operand reaches the tensor cores exactly:
+//
+// bf16 cache (kDirectBf16, 320 threads): Q, K and V stay bf16 and both
+// products run as kind::f16 MMAs with bf16 operands.  A TMA warp loads each
+// full 16-token block of a tile straight from the pools (two 64-column boxes
+// per operand, the block table giving the row); the warp itself writes the
+// rows of a block the context ends in (its valid rows, zeros after them), of
+// blocks past the context and of blocks with an out-of-range id (zeros,
+// flagged).  P = 2^(s - m) enters O += P V as a bf16 value plus its bf16
+// rounding residual (two MMAs into the same TMEM accumulator): ~16
+// significant bits, where one bf16 P would cost up to 2^-9 |v - o| on short
+// contexts.  No workspace is needed.
+//
+// fp8 cache: E4M3 values widen to f16 exactly, so the products run in f16.  A
+// bf16 query row is multiplied by the power of two 2^e that brings its largest
+// magnitude into [2^14, 2^15) before it is rounded to f16 (every element at
+// least 2^-28 of the row's largest keeps all of its bits; smaller ones keep
+// an absolute precision of 2^-39 of it), and that row's score scale is
+// multiplied by 2^-e -- exact, and free in the loop.  P is f16 (11
+// significant bits).  The operands come one of two ways:
 //
 // With a workspace (kStaged, 320 threads): prefill_widen_kernel first writes
 // each chunk's history, per kv head, as f16 rows (zeros past the context), so
 // the 16 query tiles of a 512-query chunk share one widening instead of each
-// doing its own.  Then:
-//   warps 0-7  softmax, two warps per row: warps w and w+4 own rows
-//              32 (w%4) .. +31 (TMEM lanes) and take half a key tile each;
-//              they read S from TMEM, mask, keep an online max/sum (the
-//              halves' maxima meet in shared memory at a named barrier),
-//              write P (f16) back to TMEM, rescale their half of the TMEM
-//              output only when the max grew by more than 2^8, and write the
-//              normalised output at the end;
-//   warp 8     TMEM owner and MMA issuer (one elected lane): S = Q K^T into a
-//              double-buffered TMEM score tile, O += P V into TMEM with P
-//              read from TMEM (double-buffered);
-//   warp 9     TMA producer: two 64-column boxes per operand straight from
-//              the workspace into 3 K and 2 V stages (128-byte swizzle).
+// doing its own, and a TMA warp streams two 64-column boxes per operand into
+// 3 K and 2 V stages.
 //
-// Without one (kWidenFp8 320 threads, kWidenBf16 288): one softmax warp per
-// row (warps 0-3), the MMA warp 8, and converter warps 4-7 that widen each
-// tile themselves and write both operands as [key][d] rows in the
-// 128-byte-swizzled layout (K-major for K, MN-major for V, so V needs no
-// transpose): fp8 codes exactly to f16 (K on the conversion pipe; V on the
-// integer pipe as code x 2^-8, folded into the output scale), bf16 values
-// converted to f16.  With an fp8 cache warp 9 brings each tile's raw rows
-// into a 2-stage shared-memory ring by TMA, two tiles ahead.
+// Without one (kWidenFp8, 320 threads): one softmax warp per row (warps 0-3)
+// and converter warps 4-7 that widen each tile themselves and write both
+// operands as [key][d] rows in the 128-byte-swizzled layout (K-major for K,
+// MN-major for V, so V needs no transpose): K on the conversion pipe, V on the
+// integer pipe as code x 2^-8 (folded into the output scale); warp 9 brings
+// each tile's raw rows into a 2-stage shared-memory ring by TMA, two tiles
+// ahead.
 //
-// Both MMAs run in f16 with fp32 accumulation: every E4M3 value is exact in
-// f16, bf16 inputs are exact while inside f16's range (|x| <= 65504; below
-// 2^-14 they keep an absolute precision of 2^-24), and P gets 11 significant
-// bits instead of bf16's 8.  K stages are released as soon as S = Q K^T has
-// read them, V stages once O += P V has.  S(j+1) is issued before
-// O += P(j) V(j), so the next tile's QK^T overlaps this tile's softmax.  All
-// waits are bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA
-// drains its tensor-core work and loads in flight and frees its TMEM before
-// returning.
+// Two-warps-per-row softmax (kDirectBf16, kStaged): warps w and w+4 own rows
+// 32 (w%4) .. +31 (TMEM lanes) and take half a key tile each; they read S from
+// TMEM, mask, keep an online max/sum (the halves' maxima meet in shared
+// memory at a named barrier), write P back to TMEM, rescale their half of the
+// TMEM output only when the max grew by more than 2^8, and write the
+// normalised output at the end.  Warp 8 owns TMEM and issues the MMAs from one
+// lane: S = Q K^T into a double-buffered TMEM score tile, O += P V into TMEM
+// with P read from TMEM.  K stages are released as soon as S = Q K^T has read
+// them, V stages once O += P V has.  S(j+1) is issued before O += P(j) V(j),
+// so the next tile's QK^T overlaps this tile's softmax.  All waits are
+// bounded; a wait that gives up flags PA_DEVERR_TIMEOUT, the CTA drains its
+// tensor-core work and loads in flight and frees its TMEM before returning.
 #include <type_traits>
 #include <utility>
 
@@ -60,44 +72,54 @@ namespace {
 constexpr int D = 128;       // head dim
 constexpr int BM = 128;      // rows per CTA tile
 constexpr int BN = 128;      // keys per tile
-// TMEM columns: S[2] (2 x 128 fp32), O (128 fp32), P[2] (2 x 64 columns of f16 pairs)
+// TMEM columns: S[2] (2 x 128 fp32), O (128 fp32), then P: two buffers of 64
+// columns of f16 pairs (fp8 cache), or one buffer of bf16 pairs with its
+// residual pairs in the next 64 columns (bf16 cache)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (factor 256)
 
 // Where the K/V operands come from:
-//   kWidenBf16 / kWidenFp8: warps 4-7 read the tile's rows through the block
-//     table and widen them to f16 in shared memory (with an fp8 cache a tenth
-//     warp first brings the raw rows into a 2-stage ring by TMA);
-//   kStaged: the chunk's history was widened once into an f16 workspace by
+//   kWidenFp8: warps 4-7 widen each tile's fp8 rows to f16 in shared memory,
+//     after a tenth warp has brought the raw rows into a 2-stage ring by TMA;
+//   kStaged: the chunk's fp8 history was widened once into an f16 workspace by
 //     prefill_widen_kernel (all query tiles of a chunk and kv head share it),
-//     and a TMA warp streams ready operands; there are no converter warps.
-enum Mode : int { kWidenBf16 = 0, kWidenFp8 = 1, kStaged = 2 };
+//     and a TMA warp streams ready operands; there are no converter warps;
+//   kDirectBf16: a TMA warp streams the bf16 pool's blocks themselves.
+enum Mode : int { kWidenFp8 = 0, kStaged = 1, kDirectBf16 = 2 };
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr int kOpBytes = BM * D * 2;  // one 128x128 16-bit operand = 32 KiB
 constexpr int kRawBytes = BN * D;     // one tile's fp8 K (or V) rows = 16 KiB
-constexpr int kMaxKStages = 3, kMaxVStages = 4, kRawStages = 2;
+constexpr int kMaxKStages = 3, kMaxVStages = 2, kRawStages = 2;
 template <int MODE>
 struct Layout {
-  static constexpr bool kStagedOps = MODE == kStaged;
+  static constexpr bool kTmaOps = MODE != kWidenFp8;  // operands arrive by TMA, no converters
   static constexpr bool kRawRing = MODE == kWidenFp8;
-  // staged: each row's softmax is split over two warps (8 softmax warps)
-  static constexpr bool kSplitSoftmax = kStagedOps;
-  static constexpr int kSoftWarps = kSplitSoftmax ? 8 : 4;
-  static constexpr int kMmaWarp = 8;
-  static constexpr int kLoadWarp = 9;  // none for kWidenBf16
-  static constexpr int kThreads = (kStagedOps || kRawRing) ? 320 : 288;
-  static constexpr int kKStages = kStagedOps ? 3 : 2;
-  static constexpr int kVStages = kStagedOps ? 2 : (kRawRing ? 2 : 4);
+  static constexpr bool kBf16 = MODE == kDirectBf16;  // bf16 MMAs, P as value + residual
+  static constexpr int kPBufs = kBf16 ? 1 : 2;         // P buffers in TMEM
+  // TMA-fed kernels split each row's softmax over kParts warps (4 kParts
+  // softmax warps, kParts per TMEM lane quadrant); the in-kernel widening
+  // keeps one softmax warp per quadrant and 4 converter warps
+  static constexpr bool kSplitSoftmax = kTmaOps;
+  static constexpr int kParts = kSplitSoftmax ? 4 : 1;
+  static constexpr int kSoftWarps = 4 * kParts;
+  static constexpr int kMmaWarp = kSplitSoftmax ? kSoftWarps : 8;
+  static constexpr int kLoadWarp = kMmaWarp + 1;
+  static constexpr int kThreads = (kLoadWarp + 1) * 32;
+  static constexpr int kKStages = kTmaOps ? 3 : 2;
+  static constexpr int kVStages = 2;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kOpBytes;             // K stages
   static constexpr int kVOff = kKOff + kKStages * kOpBytes;  // V stages
   static constexpr int kRawOff = kVOff + kVStages * kOpBytes;  // raw fp8 K, V stages
-  // split softmax: row maxima of the two halves [2 parities][2 halves][BM],
-  // then the halves' row sums [2][BM]
+  // split softmax: row maxima of the parts [2 parities][kParts][BM], then
+  // the parts' row sums [kParts][BM]
   static constexpr int kRedOff = kRawOff + (kRawRing ? kRawStages * 2 * kRawBytes : 0);
-  static constexpr int kBarOff = kRedOff + (kSplitSoftmax ? 6 * BM * 4 : 0);
+  // per-row score scale (scale x log2 e x the row's 2^-e) [BM]
+  static constexpr int kRowScaleOff = kRedOff + (kSplitSoftmax ? 3 * kParts * BM * 4 : 0);
+  static constexpr int kBarOff = kRowScaleOff + BM * 4;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 // 128x128 16-bit operand with the 128-byte swizzle: 128-byte rows of 64
@@ -203,6 +225,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+// KP/2 columns (KP = 32 or 64 keys as pairs) from v
+template <int KP>
+__device__ __forceinline__ void tmem_st_pairs(uint32_t taddr, const uint32_t* v) {
+  if constexpr (KP == 64)
+    tmem_st32(taddr, reinterpret_cast<const float*>(v));
+  else
+    tmem_st16(taddr, reinterpret_cast<const float*>(v));
+}
 // 2^x with the hardware approximation (relative error far below f16's 2^-11;
 // results below 2^-126 flush to zero, which P can afford)
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -237,26 +279,37 @@ __device__ __forceinline__ bool aborted(Bars* B) {
   return *reinterpret_cast<volatile int*>(&B->abort_flag) != 0;
 }
 
-// bf16x2 -> f16x2 (exact for values inside f16's normal range)
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-  return pack2<false>(f.x, f.y);
+// Rows of a block that the TMA cannot load whole (the block the context ends
+// in, blocks past the context, blocks with an out-of-range id), written by
+// the load warp into operand stage `op` at rows 16 m .. 16 m + 15: rows below
+// `nvalid` are copied from the pool row `src_row` on, the rest are zeros.
+// 16-byte chunks, eight per lane.
+__device__ __forceinline__ void write_block_rows(uint8_t* op, int m, const uint8_t* pool,
+                                                 long long src_row, int nvalid, int lane) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int idx = lane + 32 * u, r = idx >> 4, cc = idx & 15;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < nvalid)
+      v = __ldg(reinterpret_cast<const uint4*>(pool + (src_row + r) * (D * 2) + cc * 16));
+    *reinterpret_cast<uint4*>(op + op_off(16 * m + r, cc)) = v;
+  }
 }
 
 // tmk / tmv: with kWidenFp8 maps over the fp8 pools ([token rows][128]
 // bytes, 16 x 128-byte boxes); with kStaged maps over the f16 workspace
-// ([rows][128] f16, 64 x 128-element boxes); unused with kWidenBf16
+// ([rows][128] f16, 64 x 128-element boxes); with kDirectBf16 maps over the
+// bf16 pools ([token rows][128] bf16, 64 x 16-element boxes)
 template <int MODE>
 __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     prefill_tc_kernel(const PrefillParams p, const void* __restrict__ k_pool,
                       const void* __restrict__ v_pool, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   using LY = Layout<MODE>;
-  constexpr bool FP8 = MODE == kWidenFp8;
-  constexpr int kKStages = LY::kKStages, kVStages = LY::kVStages;
+  constexpr int kKStages = LY::kKStages, kVStages = LY::kVStages, kPB = LY::kPBufs;
   constexpr int kMmaWarp = LY::kMmaWarp, kLoadWarp = LY::kLoadWarp;
-  // stage "full" barriers: a TMA transaction count (staged) or the 128 converters
-  constexpr uint32_t kFullCount = LY::kStagedOps ? 1 : 128;
+  // stage "full" barriers: a TMA transaction count or the 128 converters
+  constexpr uint32_t kFullCount = LY::kTmaOps ? 1 : 128;
   constexpr int kQOff = LY::kQOff, kKOff = LY::kKOff, kVOff = LY::kVOff, kBarOff = LY::kBarOff;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -268,19 +321,43 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
   const int tile = gridDim.x - 1 - blockIdx.x, kvh = blockIdx.y, c = blockIdx.z;
   const int G = p.group;
   const int QT = BM / G;  // queries per CTA tile
-  const int q0 = p.query_start_loc[c], q1 = p.query_start_loc[c + 1];
-  const int L = q1 - q0;
-  const int ctx = p.context_lens[c];
-  if (L < 0 || L > p.max_chunk_len || ctx < L || ctx > p.max_blocks * 16) {
-    if (threadIdx.x == 0 && tile == 0 && kvh == 0) flag_error(p.dev_err, PA_DEVERR_QUERY_LOC);
-    return;
+  int q0, L, ctx;
+  if (p.fixed_q_len > 0) {
+    // multi-query decode: sequence c's fixed_q_len queries are the last
+    // positions of its context; a query before the context's start sees no
+    // key.  A context beyond the table is flagged and clamped, as in decode.
+    L = p.fixed_q_len;
+    q0 = c * L;
+    ctx = p.context_lens[c];
+    if (ctx > p.max_blocks * 16) {
+      if (threadIdx.x == 0 && tile == 0 && kvh == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+      ctx = p.max_blocks * 16;
+    }
+    ctx = max(ctx, 0);
+  } else {
+    q0 = p.query_start_loc[c];
+    L = p.query_start_loc[c + 1] - q0;
+    ctx = p.context_lens[c];
+    if (L < 0 || L > p.max_chunk_len || ctx < L || ctx > p.max_blocks * 16) {
+      if (threadIdx.x == 0 && tile == 0 && kvh == 0) flag_error(p.dev_err, PA_DEVERR_QUERY_LOC);
+      return;
+    }
   }
-  const int H = ctx - L;
+  const int H = ctx - L;  // negative only in multi-query decode
   const int i0 = tile * QT;
   if (i0 >= L) return;
   const int i_end = min(L, i0 + QT);
-  const int n_keys = H + i_end;
+  const int n_keys = max(0, H + i_end);
   const int nkt = (n_keys + BN - 1) / BN;
+  if (nkt == 0) {  // no query of this tile sees a key: all-zero rows
+    for (int idx = threadIdx.x; idx < BM * (D / 8); idx += blockDim.x) {
+      const int r = idx / (D / 8), i = i0 + r / G;
+      if (i < L)
+        reinterpret_cast<uint4*>(p.out)[((size_t)(q0 + i) * p.n_q + (size_t)kvh * G + r % G) *
+                                            (D / 8) + idx % (D / 8)] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
@@ -314,19 +391,46 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // Q tile -> shared (K-major, swizzled), one row per softmax thread
+  // Q tile -> shared (K-major, swizzled), one row per thread of warps 0-3.
+  // bf16 cache: the bf16 row as it is.  fp8 cache: the row times 2^e, e
+  // chosen from its largest magnitude, rounded to f16; the row's score scale
+  // takes the 2^-e.
+  float* row_scale = reinterpret_cast<float*>(smem + LY::kRowScaleOff);
   if (tid < BM) {
     const int r = tid, i = i0 + r / G, g = r % G;
     const bool valid = i < L;
     const uint4* src = reinterpret_cast<const uint4*>(
         reinterpret_cast<const __nv_bfloat16*>(p.q) +
         ((size_t)(q0 + (valid ? i : 0)) * p.n_q + (size_t)kvh * G + g) * D);
+    if constexpr (LY::kBf16) {
 #pragma unroll
-    for (int ch = 0; ch < 16; ++ch) {
-      uint4 v = valid ? src[ch] : make_uint4(0, 0, 0, 0);
-      v = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                     bf16x2_to_f16x2(v.w));  // the MMAs run in f16
-      *reinterpret_cast<uint4*>(smem + kQOff + op_off(r, ch)) = v;
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint4 v = valid ? src[ch] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + kQOff + op_off(r, ch)) = v;
+      }
+      row_scale[r] = p.scale_log2;
+    } else {
+      uint4 v[16];
+      uint32_t mag = 0;  // largest |x| of the row, as bf16 bits (order-preserving)
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        v[ch] = valid ? src[ch] : make_uint4(0, 0, 0, 0);
+        mag = max(mag, bf16x2_max_mag(v[ch].x));
+        mag = max(mag, bf16x2_max_mag(v[ch].y));
+        mag = max(mag, bf16x2_max_mag(v[ch].z));
+        mag = max(mag, bf16x2_max_mag(v[ch].w));
+      }
+      const int e = f16_row_shift(mag);
+      const float up = exp2i(e);
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint4 w = make_uint4(bf16x2_to_f16x2_scaled(v[ch].x, up),
+                                   bf16x2_to_f16x2_scaled(v[ch].y, up),
+                                   bf16x2_to_f16x2_scaled(v[ch].z, up),
+                                   bf16x2_to_f16x2_scaled(v[ch].w, up));
+        *reinterpret_cast<uint4*>(smem + kQOff + op_off(r, ch)) = w;
+      }
+      row_scale[r] = p.scale_log2 * exp2i(-e);
     }
     fence_async_smem();
   }
@@ -339,10 +443,12 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
   if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // kind::f16: D f32, A and B f16, N = 128, M = 128; B K-major for
-      // S = Q K^T, MN-major (bit 16) for O += P V
+      // kind::f16: D f32, N = 128, M = 128; A and B bf16 (bf16 cache) or f16
+      // (fp8 cache, and P with it); B K-major for S = Q K^T, MN-major (bit
+      // 16) for O += P V
+      constexpr uint32_t kAB = LY::kBf16 ? ((1u << 7) | (1u << 10)) : 0u;
       const uint32_t idesc =
-          (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+          (1u << 4) | kAB | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
       const uint32_t idesc_pv = idesc | (1u << 16);
       const uint32_t aQ = sbase + kQOff;
       bool ok = true;
@@ -363,16 +469,18 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           tc_commit(&B->k_empty[sk]);  // the K stage is free once S(j) is done
         }
         if (j >= 1) {  // O += P(j-1) V(j-1), P from TMEM
-          const int jp = j - 1, b = jp & 1, sv = jp % kVStages;
+          const int jp = j - 1, b = jp % kPB, sv = jp % kVStages;
           ok = wait_or_abort(&B->v_full[sv], (jp / kVStages) & 1, B, p.dev_err);
-          if (ok) ok = wait_or_abort(&B->p_full[b], (jp >> 1) & 1, B, p.dev_err);
+          if (ok) ok = wait_or_abort(&B->p_full[b], (jp / kPB) & 1, B, p.dev_err);
           if (!ok) break;
           tc_fence_after();
           const uint32_t bV = sbase + kVOff + sv * kOpBytes;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {  // 16 keys = two 8-row groups per step
-            tc_mma_ts(tO, tP + b * (BN / 2) + kk * 8, smem_desc(bV + kk * 2048, 16384),
-                      idesc_pv, (jp > 0 || kk > 0));
+            const uint64_t vd = smem_desc(bV + kk * 2048, 16384);
+            tc_mma_ts(tO, tP + b * (BN / 2) + kk * 8, vd, idesc_pv, (jp > 0 || kk > 0));
+            if constexpr (LY::kBf16)  // the residual of P, into the same accumulator
+              tc_mma_ts(tO, tP + BN / 2 + kk * 8, vd, idesc_pv, 1u);
           }
           tc_commit(&B->pv_done[b]);
           tc_commit(&B->v_empty[sv]);
@@ -383,7 +491,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       mbar_wait(&B->done, 0);
     }
   } else if (warp == kLoadWarp) {
-    if constexpr (LY::kStagedOps) {
+    if constexpr (MODE == kStaged) {
       // --------------------------------------- f16 operands from the workspace
       // Tile j of this chunk and kv head is rows row0 + 128 j .. + 127 of the
       // workspace; each operand is two 64-column boxes (its two 16 KiB halves,
@@ -424,7 +532,87 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         for (int t = max(0, issued_v - kVStages); t < issued_v; ++t)
           mbar_wait(&B->v_full[t % kVStages], (t / kVStages) & 1);
       }
-    } else if constexpr (FP8) {
+    } else if constexpr (MODE == kDirectBf16) {
+      // ------------------------------------------ bf16 blocks straight by TMA
+      // Lane m < 8 holds block m of tile j.  A whole block of the context
+      // with an id in range is two 64-column boxes per operand (rows
+      // 16 m .. 16 m + 15 of the stage's two halves), counted on the stage's
+      // full barrier.  The rows of every other block (the one the context
+      // ends in, those past it, those with an out-of-range id) the warp
+      // writes itself before that barrier's arrival, so the MMA reads them
+      // too: zeros past the context, so that 0 x garbage never reaches O.
+      const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
+      if (lane == 0) {
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
+      }
+      const uint8_t* kp = static_cast<const uint8_t*>(k_pool);
+      const uint8_t* vp = static_cast<const uint8_t*>(v_pool);
+      constexpr uint32_t kBlockBytes = 16u * D * 2u;  // one operand's rows of a block
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < nkt; ++j) {
+        const int sk = j % kKStages, sv = j % kVStages;
+        const int blk = j * 8 + lane;
+        const bool in_ctx = lane < 8 && blk * 16 < ctx;
+        const int phys = in_ctx ? __ldg(&bt[blk]) : -1;
+        const bool in_range = phys >= 0 && phys < p.num_blocks;
+        if (in_ctx && !in_range) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+        const bool whole = in_ctx && in_range && blk * 16 + 16 <= ctx;
+        const uint32_t whole_m = __ballot_sync(0xffffffffu, whole);
+        const uint32_t part_m = __ballot_sync(0xffffffffu, lane < 8 && !whole);
+        const int y = whole ? (phys * p.n_kv + kvh) * 16 : 0;  // row in the [token rows][D] view
+        // the rows of the blocks written by the warp: the valid ones, then zeros
+        auto write_parts = [&](uint8_t* op, const uint8_t* pool) {
+          for (uint32_t pm = part_m; pm; pm &= pm - 1) {
+            const int m = __ffs(pm) - 1;
+            const int ph = __shfl_sync(0xffffffffu, phys, m);
+            const bool ok_id = ph >= 0 && ph < p.num_blocks;
+            const int nvalid = ok_id ? max(0, min(16, ctx - (j * 8 + m) * 16)) : 0;
+            write_block_rows(op, m, pool, ok_id ? (long long)(ph * p.n_kv + kvh) * 16 : 0,
+                             nvalid, lane);
+          }
+          fence_async_smem();
+          __syncwarp();
+        };
+        if (j >= kKStages) {
+          const bool ok = wait_or_abort(&B->k_empty[sk], ((j - kKStages) / kKStages) & 1, B,
+                                        p.dev_err) &&
+                          !aborted(B);
+          if (!__all_sync(0xffffffffu, ok)) break;
+        }
+        uint8_t* kd = smem + kKOff + sk * kOpBytes;
+        write_parts(kd, kp);
+        if (lane == 0) mbar_arrive_expect_tx(&B->k_full[sk], __popc(whole_m) * kBlockBytes);
+        __syncwarp();
+        if (whole) {
+          tma_load_2d(kd + lane * 2048, &tmk, &B->k_full[sk], 0, y);
+          tma_load_2d(kd + kOpBytes / 2 + lane * 2048, &tmk, &B->k_full[sk], 64, y);
+        }
+        issued_k = j + 1;
+        if (j >= kVStages) {
+          const bool ok = wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1, B,
+                                        p.dev_err) &&
+                          !aborted(B);
+          if (!__all_sync(0xffffffffu, ok)) break;
+        }
+        uint8_t* vd = smem + kVOff + sv * kOpBytes;
+        write_parts(vd, vp);
+        if (lane == 0) mbar_arrive_expect_tx(&B->v_full[sv], __popc(whole_m) * kBlockBytes);
+        __syncwarp();
+        if (whole) {
+          tma_load_2d(vd + lane * 2048, &tmv, &B->v_full[sv], 0, y);
+          tma_load_2d(vd + kOpBytes / 2 + lane * 2048, &tmv, &B->v_full[sv], 64, y);
+        }
+        issued_v = j + 1;
+      }
+      // loads still in flight when the CTA gives up land before it exits
+      if (lane == 0) {
+        for (int t = max(0, issued_k - kKStages); t < issued_k; ++t)
+          mbar_wait(&B->k_full[t % kKStages], (t / kKStages) & 1);
+        for (int t = max(0, issued_v - kVStages); t < issued_v; ++t)
+          mbar_wait(&B->v_full[t % kVStages], (t / kVStages) & 1);
+      }
+    } else {
       // ----------------------------------------------- raw fp8 tiles by TMA
       // Lane m < 8 loads block m of tile t: its 16 K rows and 16 V rows of
       // 128 bytes, one box each, into raw stage t % 2 with the 128-byte
@@ -466,12 +654,11 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     }
   } else if (warp >= LY::kSoftWarps) {
     // ------------------------------------------------------------ converters
-    if constexpr (!LY::kStagedOps) {
+    if constexpr (LY::kRawRing) {
     const int ct = tid - LY::kSoftWarps * 32;  // 0..127
     const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
-    const int kv_es = FP8 ? 1 : 2;
     // block ids of a tile's 8 blocks (-1 past the context); the next tile's
-    // are loaded a tile ahead so the K/V loads never wait on the block table
+    // are loaded a tile ahead so the K/V reads never wait on the block table
     auto load_ids = [&](int j, int (&ids)[8]) {
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -486,102 +673,66 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       const int s = j % kKStages, sv = j % kVStages;
       uint8_t* kop = smem + kKOff + s * kOpBytes;
       uint8_t* vop = smem + kVOff + sv * kOpBytes;
-      // bf16: bulk-prefetch tile j+1's K and V blocks into L2, so that the
-      // loads of the next tile hit L2 instead of HBM; fp8: wait for the raw tile
-      bool raw_stop = false;
+      // wait for the raw tile
       const int rs = j % kRawStages;
       const uint8_t* raw = smem + LY::kRawOff + rs * 2 * kRawBytes;
-      if constexpr (FP8)
-        raw_stop = !wait_or_abort(&B->raw_full[rs], (j / kRawStages) & 1, B, p.dev_err);
-      if (!FP8 && j + 1 < nkt && ct < 16) {
-        const int blk = (j + 1) * 8 + (ct & 7);
-        const int phys = blk * 16 < ctx ? __ldg(&bt[blk]) : -1;
-        if (phys >= 0 && phys < p.num_blocks)
-          prefetch_l2_bulk(static_cast<const uint8_t*>(ct < 8 ? k_pool : v_pool) +
-                               ((size_t)phys * p.n_kv + kvh) * 16 * D * kv_es,
-                           16 * D * kv_es);
+      const bool raw_stop = !wait_or_abort(&B->raw_full[rs], (j / kRawStages) & 1, B, p.dev_err);
+      // Pass m covers block m of the tile: thread ct takes key ct/8, 16-byte
+      // chunk ct%8 of the stored K and V rows.  The reads of all 8 passes go
+      // out before the operand stages are released, so their latency overlaps
+      // the tensor-core work still reading them.
+      uint4 kr[8], vr[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int kib = ct >> 3;  // key in block
+        const int cc = ct & 7;    // 16-byte chunk in the row
+        const int key = j * BN + m * 16 + kib;
+        kr[m] = make_uint4(0, 0, 0, 0);
+        vr[m] = make_uint4(0, 0, 0, 0);
+        if (key < ctx) {
+          const int phys = id_cur[m];
+          if (phys < 0 || phys >= p.num_blocks) {
+            if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+          } else if (!raw_stop) {  // row kib of block m in the swizzled raw stage
+            const uint32_t ro = m * 16 * D + swz128(kib * 128 + cc * 16);
+            kr[m] = *reinterpret_cast<const uint4*>(raw + ro);
+            vr[m] = *reinterpret_cast<const uint4*>(raw + kRawBytes + ro);
+          }
+        }
       }
-      // Each pass covers 128 x 16-byte chunks of stored K and V rows: for fp8,
-      // pass m is block m of the tile (thread ct: key ct/8, chunk ct%8); for
-      // bf16, pass m is half of block m/2 (key 8(m%2) + ct/16, chunk ct%16).
-      // The loads of 8 passes go out together; the first group's before the
-      // stage is released, so their latency overlaps the tensor-core work
-      // still reading it.
-      constexpr int kPasses = FP8 ? 8 : 16;
+      // the K stage is free once S(j-2) is done, the V stage once O += P V of
+      // tile j - kVStages is
+      mbar_arrive(&B->raw_empty[rs]);  // raw tile j read
+      bool stop = raw_stop || (j >= kKStages && !wait_or_abort(&B->k_empty[s],
+                                                               ((j - kKStages) / kKStages) & 1,
+                                                               B, p.dev_err));
+      stop = stop || (j >= kVStages &&
+                      !wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1, B,
+                                     p.dev_err));
+      if (conv_bar_or(stop || aborted(B))) break;  // all converters stop together
 #pragma unroll
-      for (int g0 = 0; g0 < kPasses; g0 += 8) {
-        uint4 kr[8], vr[8];
+      for (int m = 0; m < 8; ++m) {
+        const int kib = ct >> 3, cc = ct & 7;
+        const int key_t = m * 16 + kib;  // key within tile
+        // 16 codes -> 16 f16 = 16-bit chunks 2cc, 2cc+1 (dims 16cc..16cc+15)
+        uint32_t kh[8], vh[8];
+        const uint32_t kw[4] = {kr[m].x, kr[m].y, kr[m].z, kr[m].w};
+        const uint32_t vw[4] = {vr[m].x, vr[m].y, vr[m].z, vr[m].w};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int m = g0 + u;
-          const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));  // key in block
-          const int cc = FP8 ? (ct & 7) : (ct & 15);  // 16-byte chunk in the row
-          const int key = j * BN + (FP8 ? m : (m >> 1)) * 16 + kib;
-          kr[u] = make_uint4(0, 0, 0, 0);
-          vr[u] = make_uint4(0, 0, 0, 0);
-          if (key < ctx) {
-            const int phys = id_cur[FP8 ? m : (m >> 1)];
-            if (phys < 0 || phys >= p.num_blocks) {
-              if (kib == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
-            } else if constexpr (FP8) {
-              if (!raw_stop) {  // row kib of block m in the swizzled raw stage
-                const uint32_t ro = m * 16 * D + swz128(kib * 128 + cc * 16);
-                kr[u] = *reinterpret_cast<const uint4*>(raw + ro);
-                vr[u] = *reinterpret_cast<const uint4*>(raw + kRawBytes + ro);
-              }
-            } else {
-              const size_t off = (((size_t)phys * p.n_kv + kvh) * 16 + kib) * (D * kv_es) + cc * 16;
-              kr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
-              vr[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
-            }
-          }
+        for (int e = 0; e < 4; ++e) {
+          kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
+          kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
+          vh[2 * e] = e4m3x2_to_f16x2_div256(vw[e], 0x4140u);      // codes 0, 1
+          vh[2 * e + 1] = e4m3x2_to_f16x2_div256(vw[e], 0x4342u);  // codes 2, 3
         }
-        if (g0 == 0) {  // the K stage is free once S(j-2) is done, the V stage once
-                        // O += P V of tile j - kVStages is
-          if constexpr (FP8) mbar_arrive(&B->raw_empty[rs]);  // raw tile j read
-          bool stop = raw_stop || (j >= kKStages && !wait_or_abort(&B->k_empty[s],
-                                                                   ((j - kKStages) / kKStages) & 1,
-                                                                   B, p.dev_err));
-          stop = stop || (j >= kVStages &&
-                          !wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1, B,
-                                         p.dev_err));
-          if (conv_bar_or(stop || aborted(B))) goto conv_done;  // all converters stop together
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int m = g0 + u;
-          const int kib = FP8 ? (ct >> 3) : (((m & 1) << 3) + (ct >> 4));
-          const int cc = FP8 ? (ct & 7) : (ct & 15);
-          const int key_t = (FP8 ? m : (m >> 1)) * 16 + kib;  // key within tile
-          if constexpr (FP8) {
-            // 16 codes -> 16 f16 = 16-bit chunks 2cc, 2cc+1 (dims 16cc..16cc+15)
-            uint32_t kh[8], vh[8];
-            const uint32_t kw[4] = {kr[u].x, kr[u].y, kr[u].z, kr[u].w};
-            const uint32_t vw[4] = {vr[u].x, vr[u].y, vr[u].z, vr[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
-              kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
-              vh[2 * e] = e4m3x2_to_f16x2_div256(vw[e], 0x4140u);      // codes 0, 1
-              vh[2 * e + 1] = e4m3x2_to_f16x2_div256(vw[e], 0x4342u);  // codes 2, 3
-            }
-            *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc)) =
-                make_uint4(kh[0], kh[1], kh[2], kh[3]);
-            *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc + 1)) =
-                make_uint4(kh[4], kh[5], kh[6], kh[7]);
-            *reinterpret_cast<uint4*>(vop + op_off(key_t, 2 * cc)) =
-                make_uint4(vh[0], vh[1], vh[2], vh[3]);
-            *reinterpret_cast<uint4*>(vop + op_off(key_t, 2 * cc + 1)) =
-                make_uint4(vh[4], vh[5], vh[6], vh[7]);
-          } else {
-            *reinterpret_cast<uint4*>(kop + op_off(key_t, cc)) =
-                make_uint4(bf16x2_to_f16x2(kr[u].x), bf16x2_to_f16x2(kr[u].y),
-                           bf16x2_to_f16x2(kr[u].z), bf16x2_to_f16x2(kr[u].w));
-            *reinterpret_cast<uint4*>(vop + op_off(key_t, cc)) =
-                make_uint4(bf16x2_to_f16x2(vr[u].x), bf16x2_to_f16x2(vr[u].y),
-                           bf16x2_to_f16x2(vr[u].z), bf16x2_to_f16x2(vr[u].w));
-          }
-        }
+        *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc)) =
+            make_uint4(kh[0], kh[1], kh[2], kh[3]);
+        *reinterpret_cast<uint4*>(kop + op_off(key_t, 2 * cc + 1)) =
+            make_uint4(kh[4], kh[5], kh[6], kh[7]);
+        *reinterpret_cast<uint4*>(vop + op_off(key_t, 2 * cc)) =
+            make_uint4(vh[0], vh[1], vh[2], vh[3]);
+        *reinterpret_cast<uint4*>(vop + op_off(key_t, 2 * cc + 1)) =
+            make_uint4(vh[4], vh[5], vh[6], vh[7]);
       }
       fence_async_smem();
       mbar_arrive(&B->k_full[s]);
@@ -590,67 +741,77 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       for (int m = 0; m < 8; ++m) id_cur[m] = id_nxt[m];
       if (j + 2 < nkt) load_ids(j + 2, id_nxt);  // a whole tile ahead of its first use
     }
-  conv_done:;
     }
   } else if constexpr (LY::kSplitSoftmax) {
-    // ------------------------------------------- softmax, two warps per row
-    // Warps w and w + 4 share rows 32 (w % 4) .. + 31 (the TMEM lanes warp
-    // w % 4 may access): the first takes keys 0-63 of every tile and O
-    // columns 0-63, the second keys 64-127 and O columns 64-127.  The row max
-    // of a tile is combined through shared memory at a named barrier over the
-    // 256 softmax threads, which also ORs their failure flags so that all of
-    // them leave the loop at the same barrier; the row sum is combined once at
-    // the end.  Each thread does half a row's exponentials, and two warps per
-    // sub-partition hide each other's latencies.
+    // -------------------------------------- softmax, kParts warps per row
+    // The kParts warps w, w + 4, ... share rows 32 (w % 4) .. + 31 (the TMEM
+    // lanes warp w % 4 may access); part hh takes keys KW hh .. KW hh + KW - 1
+    // of every tile and O columns OW hh .. OW hh + OW - 1.  The row max of a
+    // tile is combined through shared memory at a named barrier over all the
+    // softmax threads, which also ORs their failure flags so that all of them
+    // leave the loop at the same barrier; the row sum is combined once at the
+    // end.  Several warps per sub-partition hide each other's latencies (the
+    // TMEM loads, the exponentials, the barrier).
+    constexpr int NP = LY::kParts;
+    constexpr int KW = BN / NP;  // keys per part and tile
+    constexpr int OW = D / NP;   // O columns per part
     const int q4 = warp & 3, hh = warp >> 2;
     const int r = q4 * 32 + lane;  // row = TMEM lane
     const int i = i0 + r / G, g = r % G;
     const bool row_valid = i < L;
+    // a warp whose 32 rows are all past the chunk's queries (the tail of the
+    // last query tile; most of the tile in multi-query decode) computes no P:
+    // those rows of P and O are never read out, so it only keeps the barriers
+    const bool live = i0 + (q4 * 32) / G < L;
     const int lim = H + i;  // last visible key
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    float* red_max = reinterpret_cast<float*>(smem + LY::kRedOff);  // [2][2][BM]
-    float* red_sum = red_max + 4 * BM;                              // [2][BM]
-    const float sl = p.scale_log2;
+    float* red_max = reinterpret_cast<float*>(smem + LY::kRedOff);  // [2][NP][BM]
+    float* red_sum = red_max + 2 * NP * BM;                         // [NP][BM]
+    const float sl = row_scale[r];  // > 0 exactly when the scale is
     float m_used = -INFINITY, l = 0.f;
     bool fail = false;  // warp-uniform
+    auto load_s = [&](uint32_t ta, float* x) {
+#pragma unroll
+      for (int c32 = 0; c32 < KW / 32; ++c32) tmem_ld32(ta + c32 * 32, x + c32 * 32);
+      tmem_wait_ld();
+    };
     for (int j = 0; j < nkt; ++j) {
       const int s = j & 1;
       fail = __any_sync(0xffffffffu,
                         fail || !wait_or_abort(&B->s_full[s], (j >> 1) & 1, B, p.dev_err));
       tc_fence_after();
-      const int kbase = j * BN + hh * 64;  // first key of this half
-      const uint32_t tSrow = tS + lane_base + s * BN + hh * 64;
-      const bool full = __all_sync(0xffffffffu, row_valid && kbase + 63 <= lim) && sl > 0.f;
+      const int kbase = j * BN + hh * KW;  // first key of this part
+      const uint32_t tSrow = tS + lane_base + s * BN + hh * KW;
+      const bool full =
+          __all_sync(0xffffffffu, row_valid && kbase + KW - 1 <= lim) && p.scale_log2 > 0.f;
       float mx = -INFINITY;
-      if (!fail) {  // pass 1: this half's max
-        float x[64];
-        tmem_ld32(tSrow, x);
-        tmem_ld32(tSrow + 32, x + 32);
-        tmem_wait_ld();
+      if (!fail && live) {  // pass 1: this part's max
+        float x[KW];
+        load_s(tSrow, x);
+        float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
         if (full) {
-          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
 #pragma unroll
-          for (int e = 0; e < 64; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[e]);
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          mx *= sl;
+          for (int e = 0; e < KW; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[e]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
         } else {
-          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
+          for (int e = 0; e < KW; ++e) {
             const bool vis = !row_valid || (kbase + e <= lim);
             m4[e & 3] = fmaxf(m4[e & 3], vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
           }
           mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
       }
-      red_max[((j & 1) * 2 + hh) * BM + r] = mx;
+      float* rm = red_max + (j & 1) * NP * BM;
+      rm[hh * BM + r] = mx;
       if (named_bar_or(2, LY::kSoftWarps * 32, fail || aborted(B))) {
         fail = true;
         break;
       }
-      mx = fmaxf(mx, red_max[((j & 1) * 2 + (hh ^ 1)) * BM + r]);
+#pragma unroll
+      for (int o = 1; o < NP; ++o) mx = fmaxf(mx, rm[((hh + o) % NP) * BM + r]);
       // O and l are rescaled lazily: only when the max grew by more than 2^8;
-      // both halves of a row take the same decision
+      // all parts of a row take the same decision
       const float m_new = fmaxf(m_used, mx);
       const bool rescale = m_new > m_used + kRescaleLog2;
       float alpha = 1.f;
@@ -659,54 +820,66 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         l *= alpha;
         m_used = m_new;
       }
-      // pass 2: P = 2^(s*scale - m) as f16 pairs
+      // pass 2: P = 2^(s*scale - m) as f16 pairs, or as bf16 pairs plus the
+      // bf16 pairs of their rounding residuals
       float r4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum in 4 chains
-      uint32_t pk[32];
-      const float neg_m = -m_used;
-      {
-        float x[64];
-        tmem_ld32(tSrow, x);
-        tmem_ld32(tSrow + 32, x + 32);
-        tmem_wait_ld();
+      uint32_t pk[KW / 2], pr[LY::kBf16 ? KW / 2 : 1];
+      auto put = [&](int e, float a, float bb) {
+        if constexpr (LY::kBf16) {
+          const uint32_t h = pack2<true>(a, bb);
+          const float2 hf = unpack2<true>(h);
+          pk[e / 2] = h;
+          pr[e / 2] = pack2<true>(a - hf.x, bb - hf.y);
+        } else {
+          pk[e / 2] = pack2<false>(a, bb);
+        }
+      };
+      // a row that has seen no key yet (multi-query decode) exponentiates
+      // against 0, so that its masked scores give P = 0, not NaN
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      if (live) {
+        float x[KW];
+        load_s(tSrow, x);
         if (full) {
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
+          for (int e = 0; e < KW; e += 2) {
             const float a = fast_exp2(fmaf(x[e], sl, neg_m));
             const float bb = fast_exp2(fmaf(x[e + 1], sl, neg_m));
             r4[(e >> 1) & 3] += a + bb;
-            pk[e / 2] = pack2<false>(a, bb);
+            put(e, a, bb);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
+          for (int e = 0; e < KW; e += 2) {
             const int k0 = kbase + e;
             const float v0 = row_valid ? (k0 <= lim ? x[e] * sl : -INFINITY) : 0.f;
             const float v1 = row_valid ? (k0 + 1 <= lim ? x[e + 1] * sl : -INFINITY) : 0.f;
             const float a = fast_exp2(v0 + neg_m), bb = fast_exp2(v1 + neg_m);
             r4[(e >> 1) & 3] += a + bb;
-            pk[e / 2] = pack2<false>(a, bb);
+            put(e, a, bb);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&B->s_empty[s]);  // S buffer s may be overwritten by S(j+2)
       l += (r4[0] + r4[1]) + (r4[2] + r4[3]);
-      const int b = j & 1;
-      // P buffer b is free once O += P V of tile j-2 has completed
-      if (j >= 2)
-        fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[b], ((j - 2) >> 1) & 1, B,
+      const int b = j % kPB;
+      // P buffer b is free once O += P V of tile j - kPB has completed
+      if (j >= kPB)
+        fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[b], ((j - kPB) / kPB) & 1, B,
                                                       p.dev_err));
-      // O (this half's columns) is rescaled, rarely, once O += P V of tile j-1
-      // has completed
+      // O (this part's columns) is rescaled, rarely, once O += P V of tile
+      // j-1 has completed (with one P buffer, the wait above saw to that)
       if (!fail && j >= 1 && __any_sync(0xffffffffu, rescale)) {
-        fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[b ^ 1], ((j - 1) >> 1) & 1, B,
-                                                      p.dev_err));
+        if constexpr (kPB == 2)
+          fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[b ^ 1], ((j - 1) >> 1) & 1,
+                                                        B, p.dev_err));
         if (!fail) {
           tc_fence_after();
 #pragma unroll 1
-          for (int cc = 0; cc < 2; ++cc) {
+          for (int cc = 0; cc < OW / 32; ++cc) {
             float o[32];
-            const uint32_t ta = tO + lane_base + hh * 64 + cc * 32;
+            const uint32_t ta = tO + lane_base + hh * OW + cc * 32;
             tmem_ld32(ta, o);
             tmem_wait_ld();
 #pragma unroll
@@ -717,11 +890,15 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         }
       }
       if (!fail) {
-        tc_fence_after();
-        // column c of P buffer b holds the f16 pair (key 2c, 2c+1); this half
-        // writes columns 32 hh .. 32 hh + 31
-        tmem_st32(tP + lane_base + b * (BN / 2) + hh * 32, reinterpret_cast<const float*>(pk));
-        tmem_wait_st();
+        if (live) {
+          tc_fence_after();
+          // column c of P buffer b holds the pair (key 2c, 2c+1); this part
+          // writes columns KW/2 hh .. KW/2 hh + KW/2 - 1 (and the residuals
+          // 64 further)
+          tmem_st_pairs<KW>(tP + lane_base + b * (BN / 2) + hh * (KW / 2), pk);
+          if constexpr (LY::kBf16) tmem_st_pairs<KW>(tP + lane_base + BN / 2 + hh * (KW / 2), pr);
+          tmem_wait_st();
+        }
         tc_fence_before();
         mbar_arrive(&B->p_full[b]);
       }
@@ -729,20 +906,22 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     // epilogue: O / l after the last O += P V; every softmax thread reaches
     // this barrier once, whether the loop ended or was left together
     if (!fail)
-      fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[(nkt - 1) & 1],
-                                                    ((nkt - 1) >> 1) & 1, B, p.dev_err));
+      fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[(nkt - 1) % kPB],
+                                                    ((nkt - 1) / kPB) & 1, B, p.dev_err));
     red_sum[hh * BM + r] = l;
     if (!named_bar_or(2, LY::kSoftWarps * 32, fail)) {
       tc_fence_after();
-      const float lt = l + red_sum[(hh ^ 1) * BM + r];
+      float lt = l;
+#pragma unroll
+      for (int o = 1; o < NP; ++o) lt += red_sum[((hh + o) % NP) * BM + r];
       const float inv = (lt > 0.f) ? p.out_mul / lt : 0.f;
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) +
                            ((size_t)(q0 + (row_valid ? i : 0)) * p.n_q + (size_t)kvh * G + g) * D +
-                           hh * 64;
+                           hh * OW;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < OW / 32; ++cc) {
         float o[32];
-        tmem_ld32(tO + lane_base + hh * 64 + cc * 32, o);
+        tmem_ld32(tO + lane_base + hh * OW + cc * 32, o);
         tmem_wait_ld();
         if (row_valid) {
 #pragma unroll
@@ -762,9 +941,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     const int r = tid;  // row = TMEM lane
     const int i = i0 + r / G, g = r % G;
     const bool row_valid = i < L;
+    const bool live = i0 + (warp * 32) / G < L;  // see the split softmax
     const int lim = H + i;  // last visible key
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sl = p.scale_log2;
+    const float sl = row_scale[r];  // > 0 exactly when the scale is
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkt && ok; ++j) {
@@ -776,10 +956,12 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       const uint32_t tSrow = tS + lane_base + s * BN;
       // a tile every key of which is visible to every row of this warp needs no
       // mask: its max is taken on the raw scores (the scale is positive)
-      const bool full = __all_sync(0xffffffffu, row_valid && kbase + BN - 1 <= lim) && sl > 0.f;
+      const bool full =
+          __all_sync(0xffffffffu, row_valid && kbase + BN - 1 <= lim) && p.scale_log2 > 0.f;
       // pass 1: the row's max over this tile, 32 columns at a time
       float mx = -INFINITY;
-      if (full) {
+      if (!live) {
+      } else if (full) {
 #pragma unroll 1
         for (int cc = 0; cc < 4; cc += 2) {  // two TMEM loads in flight
           float x[64];
@@ -820,8 +1002,9 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       // buffer is free
       float r4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum in 4 chains
       uint32_t pk[BN / 2];
-      const float neg_m = -m_used;
-      if (full) {
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;  // see the split softmax
+      if (!live) {
+      } else if (full) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           float x[32];
@@ -881,11 +1064,13 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           tmem_wait_st();
         }
       }
-      tc_fence_after();
-      // P row -> TMEM: column c of buffer b holds the f16 pair (key 2c, 2c+1)
-      tmem_st32(tP + lane_base + b * (BN / 2), reinterpret_cast<const float*>(pk));
-      tmem_st32(tP + lane_base + b * (BN / 2) + 32, reinterpret_cast<const float*>(pk + 32));
-      tmem_wait_st();
+      if (live) {
+        tc_fence_after();
+        // P row -> TMEM: column c of buffer b holds the f16 pair (key 2c, 2c+1)
+        tmem_st32(tP + lane_base + b * (BN / 2), reinterpret_cast<const float*>(pk));
+        tmem_st32(tP + lane_base + b * (BN / 2) + 32, reinterpret_cast<const float*>(pk + 32));
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(&B->p_full[b]);
     }
@@ -926,15 +1111,13 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 }
 
 // ------------------------------------------------------------- widen pass
-// Writes keys 0 .. round_up(ctx_c, 128) - 1 of chunk c's history for kv head
-// h as f16 rows of the workspace: K to kst[(c n_kv + h) stage_rows + key][d],
-// V likewise to vst.  Keys at or past the context, and the keys of a block
-// whose id is out of range (flagged PA_DEVERR_BLOCK_ID), are written as
-// zeros, so the attention kernel reads finite values everywhere.  Both fp8
-// operands widen exactly (code x 1); bf16 converts to f16 as in the widening
-// kernel.  One CTA per 128-key tile; 16-byte loads and stores, a warp covering
-// whole stored rows.
-template <bool FP8>
+// Writes keys 0 .. round_up(ctx_c, 128) - 1 of chunk c's fp8 history for kv
+// head h as f16 rows of the workspace: K to kst[(c n_kv + h) stage_rows +
+// key][d], V likewise to vst.  Keys at or past the context, and the keys of a
+// block whose id is out of range (flagged PA_DEVERR_BLOCK_ID), are written as
+// zeros, so the attention kernel reads finite values everywhere.  Both
+// operands widen exactly (code x 1).  One CTA per 128-key tile; 16-byte loads
+// and stores, a warp covering whole stored rows.
 __global__ void __launch_bounds__(256)
     prefill_widen_kernel(const PrefillParams p, const void* __restrict__ k_pool,
                          const void* __restrict__ v_pool, uint16_t* __restrict__ kst,
@@ -949,8 +1132,7 @@ __global__ void __launch_bounds__(256)
   const int k0 = t * BN;
   if (k0 >= ctx) return;
   const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
-  constexpr int kES = FP8 ? 1 : 2;        // bytes per stored element
-  constexpr int kCh = D * kES / 16;       // 16-byte chunks per stored row
+  constexpr int kCh = D / 16;  // 16-byte chunks per stored fp8 row
   const size_t row0 = ((size_t)c * p.n_kv + kvh) * p.stage_rows + k0;
   for (int idx = threadIdx.x; idx < BN * kCh; idx += blockDim.x) {
     const int r = idx / kCh, cc = idx % kCh;
@@ -961,34 +1143,27 @@ __global__ void __launch_bounds__(256)
       if (phys < 0 || phys >= p.num_blocks) {
         if ((key & 15) == 0 && cc == 0) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
       } else {
-        const size_t off =
-            (((size_t)phys * p.n_kv + kvh) * 16 + (key & 15)) * (D * kES) + (size_t)cc * 16;
+        const size_t off = (((size_t)phys * p.n_kv + kvh) * 16 + (key & 15)) * D + (size_t)cc * 16;
         kr = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_pool) + off));
         vr = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_pool) + off));
       }
     }
     uint4* kd = reinterpret_cast<uint4*>(kst + (row0 + r) * D);
     uint4* vd = reinterpret_cast<uint4*>(vst + (row0 + r) * D);
-    if constexpr (FP8) {  // 16 codes -> 16 f16 (elements 16 cc .. 16 cc + 15)
-      const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w}, vw[4] = {vr.x, vr.y, vr.z, vr.w};
-      uint32_t kh[8], vh[8];
+    // 16 codes -> 16 f16 (elements 16 cc .. 16 cc + 15)
+    const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w}, vw[4] = {vr.x, vr.y, vr.z, vr.w};
+    uint32_t kh[8], vh[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
-        kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
-        vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
-        vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
-      }
-      kd[2 * cc] = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-      kd[2 * cc + 1] = make_uint4(kh[4], kh[5], kh[6], kh[7]);
-      vd[2 * cc] = make_uint4(vh[0], vh[1], vh[2], vh[3]);
-      vd[2 * cc + 1] = make_uint4(vh[4], vh[5], vh[6], vh[7]);
-    } else {
-      kd[cc] = make_uint4(bf16x2_to_f16x2(kr.x), bf16x2_to_f16x2(kr.y), bf16x2_to_f16x2(kr.z),
-                          bf16x2_to_f16x2(kr.w));
-      vd[cc] = make_uint4(bf16x2_to_f16x2(vr.x), bf16x2_to_f16x2(vr.y), bf16x2_to_f16x2(vr.z),
-                          bf16x2_to_f16x2(vr.w));
+    for (int e = 0; e < 4; ++e) {
+      kh[2 * e] = e4m3x2_to_f16x2(kw[e] & 0xffffu);
+      kh[2 * e + 1] = e4m3x2_to_f16x2(kw[e] >> 16);
+      vh[2 * e] = e4m3x2_to_f16x2(vw[e] & 0xffffu);
+      vh[2 * e + 1] = e4m3x2_to_f16x2(vw[e] >> 16);
     }
+    kd[2 * cc] = make_uint4(kh[0], kh[1], kh[2], kh[3]);
+    kd[2 * cc + 1] = make_uint4(kh[4], kh[5], kh[6], kh[7]);
+    vd[2 * cc] = make_uint4(vh[0], vh[1], vh[2], vh[3]);
+    vd[2 * cc + 1] = make_uint4(vh[4], vh[5], vh[6], vh[7]);
   }
 }
 
@@ -1034,18 +1209,14 @@ cudaError_t launch_prefill(const PrefillParams& p, pa_dtype kv_dt, const void* k
                            const void* v_pool, const CUtensorMap* tmk, const CUtensorMap* tmv,
                            void* workspace, cudaStream_t st) {
   if (p.n_chunks == 0) return cudaSuccess;
-  const bool fp8 = kv_dt == PA_FP8_E4M3;
-  if (workspace == nullptr)
-    return fp8 ? launch_tc<kWidenFp8>(p, k_pool, v_pool, tmk, tmv, st)
-               : launch_tc<kWidenBf16>(p, k_pool, v_pool, tmk, tmv, st);
+  // a bf16 cache is read as it is: no widening, no workspace
+  if (kv_dt != PA_FP8_E4M3) return launch_tc<kDirectBf16>(p, k_pool, v_pool, tmk, tmv, st);
+  if (workspace == nullptr) return launch_tc<kWidenFp8>(p, k_pool, v_pool, tmk, tmv, st);
   uint16_t* kst = static_cast<uint16_t*>(workspace);
   uint16_t* vst = kst + (size_t)p.n_chunks * p.n_kv * p.stage_rows * D;
   const dim3 grid(p.stage_rows / BN, p.n_kv, p.n_chunks);
   const cudaError_t e =
-      fp8 ? launch_dependent(prefill_widen_kernel<true>, grid, dim3(256), 0, st, p, k_pool,
-                             v_pool, kst, vst)
-          : launch_dependent(prefill_widen_kernel<false>, grid, dim3(256), 0, st, p, k_pool,
-                             v_pool, kst, vst);
+      launch_dependent(prefill_widen_kernel, grid, dim3(256), 0, st, p, k_pool, v_pool, kst, vst);
   if (e != cudaSuccess) return e;
   return launch_tc<kStaged>(p, k_pool, v_pool, tmk, tmv, st);
 }

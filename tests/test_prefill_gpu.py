@@ -4,15 +4,17 @@ Small chunks are compared in full with the oracle's causal prefill; the
 full-size mixed-step prefill (2 chunks x 512 queries over a 4096-token paged
 history, fp8 cache) is compared on sampled (query, head) rows, each of which
 the oracle computes as attention over that query's causal prefix.  Every case
-runs both ways the call can go: each query tile widening the K/V it reads,
-and with a workspace (the history widened once per chunk and kv head).  The two
-feed the tensor cores the same f16 K and V.  The workspace kernel splits each
-row's softmax over two warps (half a tile each): it decides per half whether
+runs both ways the call can go: without a workspace and with one.  With an
+fp8 cache these are two kernels (each query tile widening the K/V it reads,
+or the history widened once per chunk and kv head into the workspace) that
+feed the tensor cores the same f16 K and V; the workspace kernel splits each
+row's softmax over several warps, each deciding per part of a tile whether
 masking is needed, so an exponent argument may come from one fused
 multiply-add instead of a multiply and an add (flipping the f16 rounding of
-that P now and then), and it adds the row sum as two partial sums.  The two
-paths therefore agree to a bound far inside the oracle tolerance, not bit
-for bit.
+that P now and then), and it adds the row sum in parts.  The two fp8 paths
+therefore agree to a bound far inside the oracle tolerance, not bit for bit.
+With a bf16 cache both calls run the same kernel (bf16 operands straight from
+the pool; the workspace is not used) and agree bit for bit.
 """
 import numpy as np
 import pytest
