@@ -11,7 +11,9 @@ Prints ONE JSON line (rank 0).  `value` = decode algorithmic bytes (K and V
 of every valid context token + q + out) per second, summed over ranks, with
 inputs resident in HBM; the KV pool (~1.2 GB) is far larger than the 126 MB
 L2, so no flush is needed between steps.  Multi-GPU runs are independent
-replicas (weak scaling; decode needs no exchange between GPUs).
+replicas (weak scaling; decode needs no exchange between GPUs): under
+torchrun each rank is one GPU; `--gpus N` without a launcher starts the N
+processes itself.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
@@ -249,6 +251,80 @@ def oracle_sample_multi(inp, qm, q_len: int, budget_s: float):
 
 
 # ---------------------------------------------------------------------------
+# end-to-end staging: one pinned host buffer per step, two device buffers
+# ---------------------------------------------------------------------------
+
+class Staging:
+    """A step's host inputs packed into one pinned buffer (16-byte aligned
+    segments) and moved by ONE host-to-device copy into one of two device
+    buffers, whose segments the kernels read as typed views; outputs come back
+    by one device-to-host copy each.  Copies run on their own streams, so step
+    i+1's upload and step i's download overlap the kernels of step i."""
+
+    def __init__(self, tensors, outs, dev):
+        import torch
+        self.dev = dev
+        sizes = [t.numel() * t.element_size() for t in tensors]
+        offs, o = [], 0
+        for n in sizes:
+            offs.append(o)
+            o += (n + 15) // 16 * 16
+        self.host = torch.empty(o, dtype=torch.uint8).pin_memory()
+        for t, off, n in zip(tensors, offs, sizes):
+            self.host[off:off + n].copy_(t.detach().cpu().contiguous().view(-1).view(torch.uint8))
+        self.bufs = [torch.empty(o, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.views = [[b[off:off + n].view(t.dtype).view(t.shape)
+                       for t, off, n in zip(tensors, offs, sizes)] for b in self.bufs]
+        self.outs = [[torch.empty_like(t) for t in outs] for _ in range(2)]
+        self.outs_h = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+                       for _ in range(2)]
+        self.h2d_bytes = o
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in outs)
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()
+        self.uploaded = [ev(), ev()]
+        self.consumed = [ev(), ev()]   # kernels done with input buffer b
+        self.downloaded = [ev(), ev()]  # output buffer b copied out
+        self.used = [False, False]
+
+    def run(self, steps, kernels):
+        """`steps` pipelined steps; kernels(inputs, outputs) queues one step's
+        work on the current stream.  Returns the device time in ms, from
+        before the first upload to after the last download."""
+        import torch
+        comp = torch.cuda.current_stream(self.dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        self.up.wait_event(e0)
+        self.down.wait_event(e0)
+        self.used = [False, False]
+        for i in range(steps):
+            b = i & 1
+            if self.used[b]:
+                self.up.wait_event(self.consumed[b])
+            with torch.cuda.stream(self.up):
+                self.bufs[b].copy_(self.host, non_blocking=True)
+                self.uploaded[b].record(self.up)
+            comp.wait_event(self.uploaded[b])
+            if self.used[b]:
+                comp.wait_event(self.downloaded[b])
+            kernels(self.views[b], self.outs[b])
+            self.consumed[b].record(comp)
+            self.down.wait_event(self.consumed[b])
+            with torch.cuda.stream(self.down):
+                for dst, src in zip(self.outs_h[b], self.outs[b]):
+                    dst.copy_(src, non_blocking=True)
+                self.downloaded[b].record(self.down)
+            self.used[b] = True
+        comp.wait_stream(self.down)
+        comp.wait_stream(self.up)
+        e1.record(comp)
+        torch.cuda.synchronize(self.dev)
+        return e0.elapsed_time(e1)
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
@@ -321,48 +397,36 @@ def run_ours(args, rank, world, local):
     total_bytes = reduce_over_ranks(algo_bytes * K, "sum", world, dev)
     value = total_bytes / (ms_max / 1e3) / 1e9
 
-    # ---- end to end through the public API from pinned host buffers
-    q_h = inp.q.cpu().pin_memory()
-    key_h, val_h = key.cpu().pin_memory(), val.cpu().pin_memory()
-    slots_h = slots.cpu().pin_memory()
-    bt_h = inp.block_tables.cpu().pin_memory()
-    cl_h = inp.context_lens.cpu().pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    q_d, key_d, val_d = torch.empty_like(inp.q), torch.empty_like(key), torch.empty_like(val)
-    slots_d, bt_d, cl_d = torch.empty_like(slots), torch.empty_like(inp.block_tables), \
-        torch.empty_like(inp.context_lens)
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, key_h, val_h, slots_h, bt_h, cl_h))
-    d2h = out_h.numel() * out_h.element_size()
+    # ---- end to end through the public API from pinned host buffers: per
+    # step one upload of q, the new K/V, slots, block tables and context
+    # lengths (packed), the step's kernels, one download of the output
+    stg = Staging([inp.q, key, val, slots, inp.block_tables, inp.context_lens], [out], dev)
 
-    def e2e_step():
-        for dst, src in ((q_d, q_h), (key_d, key_h), (val_d, val_h), (slots_d, slots_h),
-                         (bt_d, bt_h), (cl_d, cl_h)):
-            dst.copy_(src, non_blocking=True)
+    def e2e_kernels(ins, outs):
+        q_d, key_d, val_d, slots_d, bt_d, cl_d = ins
         B.pa_reshape_and_cache(inp.k_pool, inp.v_pool, key_d, val_d, slots_d, inp.k_scale,
                                inp.v_scale, dev_err=err)
-        B.pa_decode(out, q_d, inp.k_pool, inp.v_pool, bt_d, cl_d, inp.scale, inp.k_scale,
+        B.pa_decode(outs[0], q_d, inp.k_pool, inp.v_pool, bt_d, cl_d, inp.scale, inp.k_scale,
                     inp.v_scale, workspace=ws, dev_err=err)
-        out_h.copy_(out, non_blocking=True)
 
     K2 = max(3, min(K, 200))
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
+    stg.run(3, e2e_kernels)
     barrier(world, dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(K2):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
+    e2e_ms = reduce_over_ranks(stg.run(K2, e2e_kernels), "max", world, dev)
     barrier(world, dev)
-    e2e_ms = reduce_over_ranks(e0.elapsed_time(e1), "max", world, dev)
     e2e_value = reduce_over_ranks(algo_bytes * K2, "sum", world, dev) / (e2e_ms / 1e3) / 1e9
+    h2d, d2h = stg.h2d_bytes, stg.d2h_bytes
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flags {int(err.item())}")
+    # the last step's downloaded output is the resident-input decode's, bit for bit
+    B.pa_decode(out, inp.q, inp.k_pool, inp.v_pool, inp.block_tables, inp.context_lens,
+                inp.scale, inp.k_scale, inp.v_scale, workspace=ws, dev_err=err)
+    if not torch.equal(stg.outs_h[(K2 - 1) & 1][0], out.cpu()):
+        raise RuntimeError("end-to-end output differs from the resident-input decode")
 
     # ---- roofline of the dominant kernel (partition kernel), live events
     kern_avg_ms = sum(kern_ms) / len(kern_ms)
+    kern_med_ms = statistics.median(kern_ms)
     peak, peak_src = hbm_peak()
     achieved = algo_bytes / (kern_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
@@ -370,6 +434,9 @@ def run_ours(args, rank, world, local):
                 "traffic": traffic_from_profile(args.workload),
                 "kernel": "decode_mma_kernel (partition kernel)",
                 "kernel_avg_us": round(kern_avg_ms * 1e3, 2),
+                "kernel_median_us": round(kern_med_ms * 1e3, 2),
+                "frac_at_median": round(algo_bytes / (kern_med_ms / 1e3) / 1e9 / peak, 4),
+                "kernel_events": len(kern_ms),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_src == "measured" else "fallback 6.65 TB/s"}
 
@@ -391,11 +458,17 @@ def run_ours(args, rank, world, local):
         "tokens_per_s": round(float(ctx.sum()) * world / (ms_max / K / 1e3), 1),
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": K2,
-                "ms_per_step": round(e2e_ms / K2, 4)},
+                "ms_per_step": round(e2e_ms / K2, 4),
+                "pipeline": "per step one packed pinned upload (q, new K/V, slots, block "
+                            "tables, context lengths) and one download of the output, on "
+                            "two copy streams double-buffered against the kernels"},
         "roofline": roofline,
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
+    if rank == 0 and args.workload == "llama3_70b_gqa_bf16" and not args.no_configs:
+        del stg
+        line["configs"] = extra_configs(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         secs, b, ns, nt, th = oracle_sample(inp, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(b / secs / 1e9, 4), "unit": "GB/s", "cores": th,
@@ -413,6 +486,135 @@ def run_ours(args, rank, world, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def tensor_peak():
+    """Measured dense bf16 burst TFLOP/s (f16 shares the nominal 2.25 PF)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (burst)"
+    except Exception:
+        return 1590.0, "fallback 1.59 PF"
+
+
+def extra_configs(dev, iters: int = 30):
+    """The other workloads' dominant kernels, each timed alone with CUDA events
+    on the launching stream (median of `iters` launches after 3 warm-ups) and
+    set against its roofline: Llama-2-7B fp16 decode, shared-prefix sampling
+    decode (L2 flushed before each call), the mixed step's fp8 decode and its
+    chunked prefill (tensor cores), and draft-token verification."""
+    import torch
+    from pagedattention_paged_kv_pa_b200 import binding as B
+    from pagedattention_paged_kv_pa_b200 import workloads as W
+    peak, psrc = hbm_peak()
+    tpeak, tsrc = tensor_peak()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+
+    def med_ms(fn, flush=False):
+        for _ in range(3):
+            fn()
+        evs = [(mk(), mk()) for _ in range(iters)]
+        for a, b in evs:
+            if flush:
+                _l2_flush(dev)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize(dev)
+        return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+    def hbm_entry(name, kernel, ms, nbytes, **kw):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        e = {"workload": name, "kernel": kernel, "median_us": round(ms * 1e3, 2),
+             "events": iters, "algorithmic_bytes": int(nbytes), "achieved": round(gbs, 1),
+             "unit": "GB/s", "peak": peak, "frac": round(gbs / peak, 4), "bound": "hbm",
+             "peak_source": psrc}
+        e.update(kw)
+        return e
+
+    res = {}
+    # Llama-2-7B fp16 decode layer and the mixed step's fp8 decode: partition kernel
+    for key, spec in (("llama2_7b_fp16", W.LLAMA2_7B_FP16),
+                      ("mixed_step_fp8_decode", W.MIXED_DECODE_FP8)):
+        inp = W.make_decode_inputs(spec, device=dev)
+        out = torch.empty_like(inp.q)
+        ws = B.alloc_decode_workspace(inp.q, inp.block_tables.shape[1])
+        ctx = inp.context_lens.cpu().numpy()
+        nbytes = W.decode_algorithmic_bytes(ctx, spec.n_q_heads, spec.n_kv_heads, spec.head_dim,
+                                            W.ELEM_BYTES[spec.q_dtype], W.ELEM_BYTES[spec.kv_dtype])
+        ms = med_ms(lambda: B.pa_decode_partitions(
+            out, inp.q, inp.k_pool, inp.v_pool, inp.block_tables, inp.context_lens, inp.scale,
+            inp.k_scale, inp.v_scale, workspace=ws, dev_err=err))
+        res[key] = hbm_entry(describe(spec, ctx, inp.num_blocks), "decode_mma_kernel", ms,
+                             nbytes, traffic=traffic_from_profile(key if key != "mixed_step_fp8_decode"
+                                                                  else "mixed_step_fp8_decode"))
+        del inp, out, ws
+    # shared-prefix sampling: one call (group + sequence partitions, merge)
+    inp, _ = W.make_shared_prefix_inputs(dev)
+    spec = inp.spec
+    ctx = inp.context_lens.cpu().numpy()
+    groups = B.prefix_groups(inp.block_tables, inp.context_lens, spec.n_q_heads,
+                             spec.n_kv_heads, spec.kv_dtype)
+    gdev = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in groups.items()}
+    out = torch.empty_like(inp.q)
+    ws = B.alloc_decode_workspace(inp.q, inp.block_tables.shape[1])
+    logical = W.decode_algorithmic_bytes(ctx, spec.n_q_heads, spec.n_kv_heads, spec.head_dim, 2, 2)
+    shared_tok = int(sum((len([m for m in row if m >= 0]) - 1) * nb * 16 for row, nb in
+                         zip(groups["members"].tolist(), groups["shared_blocks"].tolist())))
+    unique = logical - shared_tok * 2 * spec.n_kv_heads * spec.head_dim * 2
+    ms = med_ms(lambda: B.pa_decode_shared_prefix(
+        out, inp.q, inp.k_pool, inp.v_pool, inp.block_tables, inp.context_lens, inp.scale, gdev,
+        workspace=ws, dev_err=err), flush=True)
+    res["shared_prefix_bf16"] = hbm_entry(
+        "shared-prefix sampling: 16 prompts x 4 samples, bf16, 32 q / 8 kv heads",
+        "pa_decode_shared_prefix (one partition launch + merge), on unique bytes", ms, unique,
+        logical_bytes=int(logical), logical_gbs=round(logical / (ms / 1e3) / 1e9, 1),
+        l2="flushed (256 MB write) before every call")
+    del inp, out, ws
+    # draft-token verification: pa_decode_multi (partition kernel + merge)
+    spec, q_len = W.SPEC_VERIFY_BF16, W.SPEC_VERIFY_Q_LEN
+    inp = W.make_decode_inputs(spec, device=dev)
+    qm = W.make_multi_queries(inp, q_len, seed=spec.seed + 1)
+    out = torch.empty_like(qm)
+    ctx = inp.context_lens.cpu().numpy()
+    mb = inp.block_tables.shape[1]
+    ws = torch.empty(max(B.pa_decode_workspace_size(spec.num_seqs, spec.n_q_heads * q_len,
+                                                    spec.head_dim, mb), 16),
+                     dtype=torch.uint8, device=dev)
+    nbytes = (int(ctx.sum()) * 2 * spec.n_kv_heads * spec.head_dim * 2
+              + spec.num_seqs * q_len * spec.n_q_heads * spec.head_dim * 4)
+    ms = med_ms(lambda: B.pa_decode_multi(out, qm, inp.k_pool, inp.v_pool, inp.block_tables,
+                                          inp.context_lens, inp.scale, workspace=ws,
+                                          dev_err=err))
+    res["spec_verify_bf16"] = hbm_entry(describe(spec, ctx, inp.num_blocks)
+                                        + f"; {q_len} queries per sequence",
+                                        "pa_decode_multi (partition kernel + merge)", ms, nbytes,
+                                        traffic=traffic_from_profile("spec_verify_bf16"))
+    del inp, qm, out, ws
+    # the mixed step's chunked prefill: widening pass + tensor-core kernel
+    pspec = W.MIXED_PREFILL_FP8
+    pinp = W.make_prefill_inputs(pspec, device=dev)
+    pout = torch.empty_like(pinp.q)
+    pws = B.alloc_prefill_workspace(pinp.k_pool, pinp.block_tables)
+    flops = prefill_causal_flops(pinp)
+    ms = med_ms(lambda: B.pa_prefill_paged(
+        pout, pinp.q, pinp.k_pool, pinp.v_pool, pinp.block_tables, pinp.query_start_loc,
+        pinp.context_lens, pinp.scale, pspec.chunk_len, pinp.k_scale, pinp.v_scale,
+        workspace=pws, dev_err=err))
+    tf = flops / (ms / 1e3) / 1e12
+    res["mixed_step_fp8_prefill"] = {
+        "workload": "2 chunks x 512 queries over 4096-token paged histories, 32 q / 8 kv heads, "
+                    "q bf16, fp8 KV, causal", "kernel": "prefill_widen_kernel + prefill_tc_kernel",
+        "median_us": round(ms * 1e3, 2), "events": iters, "algorithmic_flop": int(flops),
+        "achieved": round(tf, 1), "unit": "TFLOP/s", "peak": tpeak, "frac": round(tf / tpeak, 4),
+        "bound": "tensor", "peak_source": tsrc}
+    del pinp, pout, pws
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flags {int(err.item())}")
+    torch.cuda.empty_cache()
+    return res
 
 
 def prefill_causal_flops(inp) -> int:
@@ -718,37 +920,21 @@ def run_spec_verify(args, rank, world, local):
     value = reduce_over_ranks(algo_bytes * K, "sum", world, dev) / (ms_max / 1e3) / 1e9
     kern_ms = sum(a.elapsed_time(b) for a, b in evs) / K
 
-    # ---- end to end through the public API from pinned host buffers
-    host = [t.cpu().pin_memory() for t in (qm, key, val, slots, inp.block_tables,
-                                            inp.context_lens)]
-    devb = [torch.empty_like(t) for t in (qm, key, val, slots, inp.block_tables,
-                                          inp.context_lens)]
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = out_h.numel() * out_h.element_size()
+    # ---- end to end through the public API: one packed upload, one download
+    stg = Staging([qm, key, val, slots, inp.block_tables, inp.context_lens], [out], dev)
 
-    def e2e_step():
-        for dst, src in zip(devb, host):
-            dst.copy_(src, non_blocking=True)
-        q_d, key_d, val_d, slots_d, bt_d, cl_d = devb
+    def e2e_kernels(ins, outs):
+        q_d, key_d, val_d, slots_d, bt_d, cl_d = ins
         B.pa_reshape_and_cache(inp.k_pool, inp.v_pool, key_d, val_d, slots_d, dev_err=err)
-        B.pa_decode_multi(out, q_d, inp.k_pool, inp.v_pool, bt_d, cl_d, inp.scale,
+        B.pa_decode_multi(outs[0], q_d, inp.k_pool, inp.v_pool, bt_d, cl_d, inp.scale,
                           workspace=ws, dev_err=err)
-        out_h.copy_(out, non_blocking=True)
 
     K2 = max(3, min(K, 200))
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
+    stg.run(3, e2e_kernels)
     barrier(world, dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(K2):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
+    e2e_ms = reduce_over_ranks(stg.run(K2, e2e_kernels), "max", world, dev)
     barrier(world, dev)
-    e2e_ms = reduce_over_ranks(e0.elapsed_time(e1), "max", world, dev)
+    h2d, d2h = stg.h2d_bytes, stg.d2h_bytes
     e2e_value = reduce_over_ranks(algo_bytes * K2, "sum", world, dev) / (e2e_ms / 1e3) / 1e9
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flags {int(err.item())}")
@@ -769,7 +955,9 @@ def run_spec_verify(args, rank, world, local):
                    "parallelism": f"replicas x{world}"},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": K2,
-                "ms_per_step": round(e2e_ms / K2, 4)},
+                "ms_per_step": round(e2e_ms / K2, 4),
+                "pipeline": "one packed pinned upload and one download per step on two copy "
+                            "streams, double-buffered against the kernels"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": traffic_from_profile("spec_verify_bf16"),
@@ -1011,7 +1199,7 @@ def run_swap(args, rank, world, local):
         dist.destroy_process_group()
 
 
-def run_alloc_host(args):
+def run_alloc_host(args, rank=0, world=1):
     """Host allocator under a synthetic serving trace (no GPU): requests drawn
     from 8 shared system prompts (256-1024 tokens) plus 16-256 private tokens
     are admitted with prefix caching on, decode 32 tokens one at a time, and
@@ -1019,6 +1207,7 @@ def run_alloc_host(args):
     are evicted under pressure.  Reports allocator calls per second and the
     share of prompt tokens whose prefill the cache saved."""
     from pagedattention_paged_kv_pa_b200 import binding as B
+    dist_init(world, "gloo")  # host-only replicas: the scalars go over gloo
     rng = np.random.default_rng(1007)
     prompts = [rng.integers(0, 1 << 30, size=int(rng.integers(256, 1025))).tolist()
                for _ in range(8)]
@@ -1050,16 +1239,44 @@ def run_alloc_host(args):
             calls += 1
             running.remove(r)
     secs = time.perf_counter() - t0
+    # replicas: every rank runs the trace; calls summed over the slowest rank's time
+    secs_max = reduce_over_ranks(secs, "max", world)
+    calls_all = reduce_over_ranks(calls, "sum", world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
     print(json.dumps({
-        "metric": "host block allocator calls/s (prefix caching on)", "value": round(calls / secs),
-        "unit": "calls/s", "n_gpus": 0, "steps": n_req, "warmup": 0,
+        "metric": "host block allocator calls/s (prefix caching on)",
+        "value": round(calls_all / secs_max), "unit": "calls/s", "n_gpus": 0, "ranks": world,
+        "scaling": "weak", "steps": n_req, "warmup": 0,
         "higher_is_better": True, "data": "synthetic serving trace (seeded)",
         "config": {"workload": "8 shared prompts of 256-1024 tokens + 16-256 private tokens, "
                                "32 decode tokens per request, <= 64 running, 6000-block pool",
                    "requests": n_req},
         "prompt_tokens_saved": round(cached_toks / max(prompt_toks, 1), 4),
-        "us_per_call": round(secs / calls * 1e6, 3), "cores": 1,
+        "us_per_call": round(secs / calls * 1e6, 3), "cores": world,
         "note": "includes the Python binding's marshalling of every call"}), flush=True)
+
+
+def spawn_replicas(n: int, argv) -> int:
+    """`--gpus N` without a launcher: start N copies of this script, one per
+    GPU (RANK = LOCAL_RANK = i, WORLD_SIZE = N, rendezvous on 127.0.0.1), as
+    torchrun would; rank 0 prints the job's line.  Returns the worst exit
+    code."""
+    import socket
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n),
+                   LOCAL_WORLD_SIZE=str(n), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, os.path.abspath(__file__)] + list(argv),
+                                      env=env))
+    return max(p.wait() for p in procs)
 
 
 def main(argv=None):
@@ -1071,8 +1288,16 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama3_70b_gqa_bf16")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' kernel rooflines in the default line")
     args = ap.parse_args(argv)
     rank, world, local = dist_env()
+    if "WORLD_SIZE" in os.environ:
+        if args.gpus != world:
+            sys.stderr.write(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}\n")
+            return 2
+    elif args.gpus > 1:
+        return spawn_replicas(args.gpus, sys.argv[1:] if argv is None else argv)
     if args.impl == "reference":
         run_reference(args, rank, world, local)
     elif args.workload == "mixed_step_fp8":
@@ -1080,14 +1305,15 @@ def main(argv=None):
     elif args.workload == "spec_verify_bf16":
         run_spec_verify(args, rank, world, local)
     elif args.workload == "alloc_host":
-        run_alloc_host(args)
+        run_alloc_host(args, rank, world)
     elif args.workload == "swap_bf16":
         run_swap(args, rank, world, local)
     elif args.workload == "shared_prefix_bf16":
         run_shared_prefix(args, rank, world, local)
     else:
         run_ours(args, rank, world, local)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())
