@@ -101,11 +101,21 @@ struct Layout {
   // softmax warps, kParts per TMEM lane quadrant); the in-kernel widening
   // keeps one softmax warp per quadrant and 4 converter warps
   static constexpr bool kSplitSoftmax = kTmaOps;
-  static constexpr int kParts = kSplitSoftmax ? 4 : 1;
+  // parts per row: the length of a softmax warp's chain per tile is what
+  // bounds it.  bf16 (also multi-query decode, whose few rows fill only
+  // two TMEM lane quadrants, i.e. two of the four SM sub-partitions): 4
+  // parts of 32 keys; fp8 from the workspace (all quadrants busy): 2 of 64,
+  // which measured faster than 4 there
+  static constexpr int kParts = !kSplitSoftmax ? 1 : (kBf16 ? 4 : 2);
   static constexpr int kSoftWarps = 4 * kParts;
   static constexpr int kMmaWarp = kSplitSoftmax ? kSoftWarps : 8;
+  // K and V are loaded by one warp, or (kSplitLoads) by two, so that K runs
+  // ahead of V, whose stages free up only after O += P V; a 19th warp would
+  // cut the registers a thread may hold below what the softmax needs
+  static constexpr bool kSplitLoads = kTmaOps && kParts < 4;
   static constexpr int kLoadWarp = kMmaWarp + 1;
-  static constexpr int kThreads = (kLoadWarp + 1) * 32;
+  static constexpr int kVLoadWarp = kSplitLoads ? kLoadWarp + 1 : kLoadWarp;
+  static constexpr int kThreads = (kVLoadWarp + 1) * 32;
   static constexpr int kKStages = kTmaOps ? 3 : 2;
   static constexpr int kVStages = 2;
   static constexpr int kQOff = 0;
@@ -490,126 +500,106 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       tc_commit(&B->done);
       mbar_wait(&B->done, 0);
     }
-  } else if (warp == kLoadWarp) {
-    if constexpr (MODE == kStaged) {
-      // --------------------------------------- f16 operands from the workspace
-      // Tile j of this chunk and kv head is rows row0 + 128 j .. + 127 of the
-      // workspace; each operand is two 64-column boxes (its two 16 KiB halves,
-      // 128-byte swizzled), counted on the stage's full barrier.
-      if (lane == 0) {
-        prefetch_tensormap(&tmk);
-        prefetch_tensormap(&tmv);
-        // launched as a programmatic dependent of the widening pass: the
-        // prologue above overlapped it; the workspace is read only after it
-        // has completed
-        pdl_wait();
-        const int row0 = (c * p.n_kv + kvh) * p.stage_rows;
-        int issued_k = 0, issued_v = 0;
-        for (int j = 0; j < nkt; ++j) {
-          const int sk = j % kKStages, sv = j % kVStages;
-          if (j >= kKStages && !(wait_or_abort(&B->k_empty[sk], ((j - kKStages) / kKStages) & 1,
-                                               B, p.dev_err) &&
-                                 !aborted(B)))
-            break;
-          uint8_t* kd = smem + kKOff + sk * kOpBytes;
-          mbar_arrive_expect_tx(&B->k_full[sk], kOpBytes);
-          tma_load_2d(kd, &tmk, &B->k_full[sk], 0, row0 + j * BN);
-          tma_load_2d(kd + kOpBytes / 2, &tmk, &B->k_full[sk], 64, row0 + j * BN);
-          issued_k = j + 1;
-          if (j >= kVStages && !(wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1,
-                                               B, p.dev_err) &&
-                                 !aborted(B)))
-            break;
-          uint8_t* vd = smem + kVOff + sv * kOpBytes;
-          mbar_arrive_expect_tx(&B->v_full[sv], kOpBytes);
-          tma_load_2d(vd, &tmv, &B->v_full[sv], 0, row0 + j * BN);
-          tma_load_2d(vd + kOpBytes / 2, &tmv, &B->v_full[sv], 64, row0 + j * BN);
-          issued_v = j + 1;
-        }
-        // loads still in flight when the CTA gives up land before it exits
-        for (int t = max(0, issued_k - kKStages); t < issued_k; ++t)
-          mbar_wait(&B->k_full[t % kKStages], (t / kKStages) & 1);
-        for (int t = max(0, issued_v - kVStages); t < issued_v; ++t)
-          mbar_wait(&B->v_full[t % kVStages], (t / kVStages) & 1);
-      }
-    } else if constexpr (MODE == kDirectBf16) {
-      // ------------------------------------------ bf16 blocks straight by TMA
-      // Lane m < 8 holds block m of tile j.  A whole block of the context
-      // with an id in range is two 64-column boxes per operand (rows
-      // 16 m .. 16 m + 15 of the stage's two halves), counted on the stage's
-      // full barrier.  The rows of every other block (the one the context
-      // ends in, those past it, those with an out-of-range id) the warp
-      // writes itself before that barrier's arrival, so the MMA reads them
-      // too: zeros past the context, so that 0 x garbage never reaches O.
+  } else if (warp == kLoadWarp || warp == LY::kVLoadWarp) {
+    if constexpr (LY::kTmaOps) {
+      // TMA-fed operands.  With split loads warp kLoadWarp loads K and warp
+      // kVLoadWarp V, so that K runs ahead of V; otherwise the load warp
+      // takes K then V of each tile.  issue(j, v) loads operand v of tile j
+      // into its stage once the stage is free; false when the CTA gives up.
       const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
+      int issued[2] = {0, 0};
       if (lane == 0) {
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
       }
-      const uint8_t* kp = static_cast<const uint8_t*>(k_pool);
-      const uint8_t* vp = static_cast<const uint8_t*>(v_pool);
-      constexpr uint32_t kBlockBytes = 16u * D * 2u;  // one operand's rows of a block
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < nkt; ++j) {
-        const int sk = j % kKStages, sv = j % kVStages;
-        const int blk = j * 8 + lane;
-        const bool in_ctx = lane < 8 && blk * 16 < ctx;
-        const int phys = in_ctx ? __ldg(&bt[blk]) : -1;
-        const bool in_range = phys >= 0 && phys < p.num_blocks;
-        if (in_ctx && !in_range) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
-        const bool whole = in_ctx && in_range && blk * 16 + 16 <= ctx;
-        const uint32_t whole_m = __ballot_sync(0xffffffffu, whole);
-        const uint32_t part_m = __ballot_sync(0xffffffffu, lane < 8 && !whole);
-        const int y = whole ? (phys * p.n_kv + kvh) * 16 : 0;  // row in the [token rows][D] view
-        // the rows of the blocks written by the warp: the valid ones, then zeros
-        auto write_parts = [&](uint8_t* op, const uint8_t* pool) {
+      // launched as a programmatic dependent of the widening pass: the
+      // prologue above overlapped it; the workspace is read only after it
+      // has completed (a no-op for other launches)
+      if (MODE == kStaged) pdl_wait();
+      auto issue = [&](int j, bool vop) -> bool {
+        const int NS = vop ? kVStages : kKStages;
+        const int st = j % NS;
+        uint64_t* full = vop ? &B->v_full[st] : &B->k_full[st];
+        uint64_t* empty = vop ? &B->v_empty[st] : &B->k_empty[st];
+        const CUtensorMap* map = vop ? &tmv : &tmk;
+        uint8_t* d = smem + (vop ? kVOff : kKOff) + st * kOpBytes;
+        if constexpr (MODE == kStaged) {
+          // tile j of this chunk and kv head is rows row0 + 128 j .. + 127 of
+          // the workspace; an operand is two 64-column boxes (its two 16 KiB
+          // halves, 128-byte swizzled), counted on the stage's full barrier
+          int ok = 1;
+          if (lane == 0) {
+            if (j >= NS)
+              ok = wait_or_abort(empty, ((j - NS) / NS) & 1, B, p.dev_err) && !aborted(B);
+            if (ok) {
+              const int row = (c * p.n_kv + kvh) * p.stage_rows + j * BN;
+              mbar_arrive_expect_tx(full, kOpBytes);
+              tma_load_2d(d, map, full, 0, row);
+              tma_load_2d(d + kOpBytes / 2, map, full, 64, row);
+            }
+          }
+          return __shfl_sync(0xffffffffu, ok, 0) != 0;
+        } else {
+          // bf16 blocks straight from the pool: lane m < 8 holds block m of
+          // tile j.  A whole block of the context with an id in range is two
+          // 64-column boxes (rows 16 m .. 16 m + 15 of the stage's halves),
+          // counted on the stage's full barrier; the rows of every other
+          // block (the one the context ends in, those past it, those with an
+          // out-of-range id) the warp writes itself before that barrier's
+          // arrival, so the MMA reads them too: zeros past the context, so
+          // that 0 x garbage never reaches O.
+          constexpr uint32_t kBlockBytes = 16u * D * 2u;  // one operand's rows of a block
+          const int blk = j * 8 + lane;
+          const bool in_ctx = lane < 8 && blk * 16 < ctx;
+          const int phys = in_ctx ? __ldg(&bt[blk]) : -1;
+          const bool in_range = phys >= 0 && phys < p.num_blocks;
+          if (!vop && in_ctx && !in_range) flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
+          const bool whole = in_ctx && in_range && blk * 16 + 16 <= ctx;
+          const uint32_t whole_m = __ballot_sync(0xffffffffu, whole);
+          const uint32_t part_m = __ballot_sync(0xffffffffu, lane < 8 && !whole);
+          const int y = whole ? (phys * p.n_kv + kvh) * 16 : 0;  // row in the [rows][D] view
+          if (j >= NS) {
+            const bool ok =
+                wait_or_abort(empty, ((j - NS) / NS) & 1, B, p.dev_err) && !aborted(B);
+            if (!__all_sync(0xffffffffu, ok)) return false;
+          }
+          const uint8_t* pool = static_cast<const uint8_t*>(vop ? v_pool : k_pool);
           for (uint32_t pm = part_m; pm; pm &= pm - 1) {
             const int m = __ffs(pm) - 1;
             const int ph = __shfl_sync(0xffffffffu, phys, m);
             const bool ok_id = ph >= 0 && ph < p.num_blocks;
             const int nvalid = ok_id ? max(0, min(16, ctx - (j * 8 + m) * 16)) : 0;
-            write_block_rows(op, m, pool, ok_id ? (long long)(ph * p.n_kv + kvh) * 16 : 0,
+            write_block_rows(d, m, pool, ok_id ? (long long)(ph * p.n_kv + kvh) * 16 : 0,
                              nvalid, lane);
           }
           fence_async_smem();
           __syncwarp();
-        };
-        if (j >= kKStages) {
-          const bool ok = wait_or_abort(&B->k_empty[sk], ((j - kKStages) / kKStages) & 1, B,
-                                        p.dev_err) &&
-                          !aborted(B);
-          if (!__all_sync(0xffffffffu, ok)) break;
+          if (lane == 0) mbar_arrive_expect_tx(full, __popc(whole_m) * kBlockBytes);
+          __syncwarp();
+          if (whole) {
+            tma_load_2d(d + lane * 2048, map, full, 0, y);
+            tma_load_2d(d + kOpBytes / 2 + lane * 2048, map, full, 64, y);
+          }
+          return true;
         }
-        uint8_t* kd = smem + kKOff + sk * kOpBytes;
-        write_parts(kd, kp);
-        if (lane == 0) mbar_arrive_expect_tx(&B->k_full[sk], __popc(whole_m) * kBlockBytes);
-        __syncwarp();
-        if (whole) {
-          tma_load_2d(kd + lane * 2048, &tmk, &B->k_full[sk], 0, y);
-          tma_load_2d(kd + kOpBytes / 2 + lane * 2048, &tmk, &B->k_full[sk], 64, y);
+      };
+      const bool only_v = LY::kSplitLoads && warp == LY::kVLoadWarp;
+      const bool only_k = LY::kSplitLoads && warp == kLoadWarp;
+      for (int j = 0; j < nkt; ++j) {
+        if (!only_v) {
+          if (!issue(j, false)) break;
+          issued[0] = j + 1;
         }
-        issued_k = j + 1;
-        if (j >= kVStages) {
-          const bool ok = wait_or_abort(&B->v_empty[sv], ((j - kVStages) / kVStages) & 1, B,
-                                        p.dev_err) &&
-                          !aborted(B);
-          if (!__all_sync(0xffffffffu, ok)) break;
+        if (!only_k) {
+          if (!issue(j, true)) break;
+          issued[1] = j + 1;
         }
-        uint8_t* vd = smem + kVOff + sv * kOpBytes;
-        write_parts(vd, vp);
-        if (lane == 0) mbar_arrive_expect_tx(&B->v_full[sv], __popc(whole_m) * kBlockBytes);
-        __syncwarp();
-        if (whole) {
-          tma_load_2d(vd + lane * 2048, &tmv, &B->v_full[sv], 0, y);
-          tma_load_2d(vd + kOpBytes / 2 + lane * 2048, &tmv, &B->v_full[sv], 64, y);
-        }
-        issued_v = j + 1;
       }
       // loads still in flight when the CTA gives up land before it exits
       if (lane == 0) {
-        for (int t = max(0, issued_k - kKStages); t < issued_k; ++t)
+        for (int t = max(0, issued[0] - kKStages); t < issued[0]; ++t)
           mbar_wait(&B->k_full[t % kKStages], (t / kKStages) & 1);
-        for (int t = max(0, issued_v - kVStages); t < issued_v; ++t)
+        for (int t = max(0, issued[1] - kVStages); t < issued[1]; ++t)
           mbar_wait(&B->v_full[t % kVStages], (t / kVStages) & 1);
       }
     } else {
@@ -785,8 +775,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       const bool full =
           __all_sync(0xffffffffu, row_valid && kbase + KW - 1 <= lim) && p.scale_log2 > 0.f;
       float mx = -INFINITY;
+      // this part's scores, read from TMEM once: the loads are slow while the
+      // tensor core works on the same TMEM, so pass 2 reuses the registers
+      float x[KW];
       if (!fail && live) {  // pass 1: this part's max
-        float x[KW];
         load_s(tSrow, x);
         float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
         if (full) {
@@ -823,13 +815,14 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       // pass 2: P = 2^(s*scale - m) as f16 pairs, or as bf16 pairs plus the
       // bf16 pairs of their rounding residuals
       float r4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum in 4 chains
-      uint32_t pk[KW / 2], pr[LY::kBf16 ? KW / 2 : 1];
+      // (the residual pairs go to x[0 .. KW/2), scores already consumed)
+      uint32_t pk[KW / 2];
       auto put = [&](int e, float a, float bb) {
         if constexpr (LY::kBf16) {
           const uint32_t h = pack2<true>(a, bb);
           const float2 hf = unpack2<true>(h);
           pk[e / 2] = h;
-          pr[e / 2] = pack2<true>(a - hf.x, bb - hf.y);
+          x[e / 2] = __uint_as_float(pack2<true>(a - hf.x, bb - hf.y));
         } else {
           pk[e / 2] = pack2<false>(a, bb);
         }
@@ -838,8 +831,6 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       // against 0, so that its masked scores give P = 0, not NaN
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       if (live) {
-        float x[KW];
-        load_s(tSrow, x);
         if (full) {
 #pragma unroll
           for (int e = 0; e < KW; e += 2) {
@@ -896,7 +887,9 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           // writes columns KW/2 hh .. KW/2 hh + KW/2 - 1 (and the residuals
           // 64 further)
           tmem_st_pairs<KW>(tP + lane_base + b * (BN / 2) + hh * (KW / 2), pk);
-          if constexpr (LY::kBf16) tmem_st_pairs<KW>(tP + lane_base + BN / 2 + hh * (KW / 2), pr);
+          if constexpr (LY::kBf16)
+            tmem_st_pairs<KW>(tP + lane_base + BN / 2 + hh * (KW / 2),
+                              reinterpret_cast<const uint32_t*>(x));
           tmem_wait_st();
         }
         tc_fence_before();
