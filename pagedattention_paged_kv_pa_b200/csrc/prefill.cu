@@ -109,13 +109,10 @@ struct Layout {
   static constexpr int kParts = !kSplitSoftmax ? 1 : (kBf16 ? 4 : 2);
   static constexpr int kSoftWarps = 4 * kParts;
   static constexpr int kMmaWarp = kSplitSoftmax ? kSoftWarps : 8;
-  // K and V are loaded by one warp, or (kSplitLoads) by two, so that K runs
-  // ahead of V, whose stages free up only after O += P V; a 19th warp would
-  // cut the registers a thread may hold below what the softmax needs
-  static constexpr bool kSplitLoads = kTmaOps && kParts < 4;
+  // one load warp takes K then V of each tile (a second warp for V measured
+  // no faster, and with 4 parts it would cut the registers a thread may hold)
   static constexpr int kLoadWarp = kMmaWarp + 1;
-  static constexpr int kVLoadWarp = kSplitLoads ? kLoadWarp + 1 : kLoadWarp;
-  static constexpr int kThreads = (kVLoadWarp + 1) * 32;
+  static constexpr int kThreads = (kLoadWarp + 1) * 32;
   static constexpr int kKStages = kTmaOps ? 3 : 2;
   static constexpr int kVStages = 2;
   static constexpr int kQOff = 0;
@@ -500,12 +497,11 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       tc_commit(&B->done);
       mbar_wait(&B->done, 0);
     }
-  } else if (warp == kLoadWarp || warp == LY::kVLoadWarp) {
+  } else if (warp == kLoadWarp) {
     if constexpr (LY::kTmaOps) {
-      // TMA-fed operands.  With split loads warp kLoadWarp loads K and warp
-      // kVLoadWarp V, so that K runs ahead of V; otherwise the load warp
-      // takes K then V of each tile.  issue(j, v) loads operand v of tile j
-      // into its stage once the stage is free; false when the CTA gives up.
+      // TMA-fed operands: K then V of each tile.  issue(j, v) loads operand v
+      // of tile j into its stage once the stage is free; false when the CTA
+      // gives up.
       const int32_t* bt = p.block_tables + (size_t)c * p.max_blocks;
       int issued[2] = {0, 0};
       if (lane == 0) {
@@ -583,17 +579,11 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
           return true;
         }
       };
-      const bool only_v = LY::kSplitLoads && warp == LY::kVLoadWarp;
-      const bool only_k = LY::kSplitLoads && warp == kLoadWarp;
       for (int j = 0; j < nkt; ++j) {
-        if (!only_v) {
-          if (!issue(j, false)) break;
-          issued[0] = j + 1;
-        }
-        if (!only_k) {
-          if (!issue(j, true)) break;
-          issued[1] = j + 1;
-        }
+        if (!issue(j, false)) break;
+        issued[0] = j + 1;
+        if (!issue(j, true)) break;
+        issued[1] = j + 1;
       }
       // loads still in flight when the CTA gives up land before it exits
       if (lane == 0) {
