@@ -379,19 +379,26 @@ def run_ours(args, rank, world, local):
     sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
     time.sleep(0.3)
     K = args.steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
+    # the timed steps carry no events between their kernels (an event record
+    # between two programmatically dependent launches costs their overlap)
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, dev)
     torch.cuda.synchronize()
     t_start.record()
     for i in range(K):
-        step(*evs[i])
+        step()
     t_stop.record()
     torch.cuda.synchronize()
     barrier(world, dev)
     clocks = sampler.stop()
     ms_total = t_start.elapsed_time(t_stop)
+    # the partition kernel alone: events around it, in a second loop of steps
+    KE = max(3, min(K, 200))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(KE)]
+    for i in range(KE):
+        step(*evs[i])
+    torch.cuda.synchronize()
     kern_ms = [a.elapsed_time(b) for a, b in evs]
     ms_max = reduce_over_ranks(ms_total, "max", world, dev)
     total_bytes = reduce_over_ranks(algo_bytes * K, "sum", world, dev)
@@ -437,6 +444,8 @@ def run_ours(args, rank, world, local):
                 "kernel_median_us": round(kern_med_ms * 1e3, 2),
                 "frac_at_median": round(algo_bytes / (kern_med_ms / 1e3) / 1e9 / peak, 4),
                 "kernel_events": len(kern_ms),
+                "kernel_timing": "events around the partition kernel in a separate loop of "
+                                 "the same steps, after the timed loop",
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_src == "measured" else "fallback 6.65 TB/s"}
 
@@ -589,8 +598,9 @@ def extra_configs(dev, iters: int = 30):
                                           dev_err=err))
     res["spec_verify_bf16"] = hbm_entry(describe(spec, ctx, inp.num_blocks)
                                         + f"; {q_len} queries per sequence",
-                                        "pa_decode_multi (partition kernel + merge)", ms, nbytes,
-                                        traffic=traffic_from_profile("spec_verify_bf16"))
+                                        "pa_decode_multi: prefill_tc_kernel (bf16 tensor cores)",
+                                        ms, nbytes,
+                                        traffic=traffic_from_profile("spec_verify_bf16", "prefill"))
     del inp, qm, out, ws
     # the mixed step's chunked prefill: widening pass + tensor-core kernel
     pspec = W.MIXED_PREFILL_FP8
@@ -608,7 +618,8 @@ def extra_configs(dev, iters: int = 30):
                     "q bf16, fp8 KV, causal", "kernel": "prefill_widen_kernel + prefill_tc_kernel",
         "median_us": round(ms * 1e3, 2), "events": iters, "algorithmic_flop": int(flops),
         "achieved": round(tf, 1), "unit": "TFLOP/s", "peak": tpeak, "frac": round(tf / tpeak, 4),
-        "bound": "tensor", "peak_source": tsrc}
+        "bound": "tensor", "peak_source": tsrc,
+        "traffic": traffic_from_profile("mixed_step_fp8_prefill", "prefill")}
     del pinp, pout, pws
     torch.cuda.synchronize(dev)
     if int(err.item()) != 0:
@@ -784,29 +795,37 @@ def run_mixed(args, rank, world, local):
 
 
 DECODE_SOURCES = ("decode.cu", "pa_internal.h", "pa_device.cuh")
+PREFILL_SOURCES = ("prefill.cu", "pa_internal.h", "pa_device.cuh")
 
 
-def decode_source_hash():
-    """First 16 hex digits of the SHA-256 of the decode kernel's sources."""
+def source_hash(files=DECODE_SOURCES):
+    """First 16 hex digits of the SHA-256 of a kernel's sources."""
     import hashlib
     h = hashlib.sha256()
-    for f in DECODE_SOURCES:
+    for f in files:
         h.update(open(os.path.join(ROOT, "pagedattention_paged_kv_pa_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile(workload):
-    """DRAM bytes per launch of the partition kernel from the committed ncu
-    summary (profiles/decode_traffic.txt), if that summary was taken on the
-    current kernel sources; None otherwise."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+def decode_source_hash():
+    return source_hash(DECODE_SOURCES)
+
+
+def traffic_from_profile(workload, kernel="decode"):
+    """DRAM bytes per launch of the decode partition kernel (kernel="decode",
+    profiles/decode_traffic.txt) or of the tensor-core prefill kernel
+    (kernel="prefill", profiles/prefill_traffic.txt) from the committed ncu
+    summaries, if they were taken on the current kernel sources; None
+    otherwise."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    files = DECODE_SOURCES if kernel == "decode" else PREFILL_SOURCES
     try:
         rec = {}
         for line in open(path):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 rec[k.strip()] = v.strip()
-        if rec.get("decode_src_sha256_16") != decode_source_hash():
+        if rec.get(f"{kernel}_src_sha256_16") != source_hash(files):
             return None
         return int(rec[workload]) if workload in rec else None
     except Exception:
@@ -960,11 +979,12 @@ def run_spec_verify(args, rank, world, local):
                             "streams, double-buffered against the kernels"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": traffic_from_profile("spec_verify_bf16"),
-                     "kernel": "pa_decode_multi (partition kernel + merge kernel)",
+                     "traffic": traffic_from_profile("spec_verify_bf16", "prefill"),
+                     "kernel": "pa_decode_multi: prefill_tc_kernel (bf16 tensor cores, one "
+                               "tile per sequence and kv head)",
                      "kernel_avg_us": round(kern_ms * 1e3, 2),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 2 * K,  # slot write + the tensor-core kernel
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1037,6 +1057,7 @@ def run_shared_prefix(args, rank, world, local):
     torch.cuda.synchronize()
     props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(f"GPU-{props.uuid}" if hasattr(props, "uuid") else str(local))
+    time.sleep(0.3)
     K = args.steps
     barrier(world, dev)
     ms = reduce_over_ranks(timed(True, K), "max", world, dev)
