@@ -107,6 +107,11 @@ struct Layout {
   // parts of 32 keys; fp8 from the workspace (all quadrants busy): 2 of 64,
   // which measured faster than 4 there
   static constexpr int kParts = !kSplitSoftmax ? 1 : (kBf16 ? 4 : 2);
+  // two parts per row keep independent softmax states, each with its own O
+  // accumulator (the two 128-column O tiles take the TMEM the P buffers had;
+  // P goes over the part's own S columns), so no per-tile max exchange ties
+  // the row's two warps together; they merge once at the end
+  static constexpr bool kIndep = kSplitSoftmax && kParts == 2;
   static constexpr int kSoftWarps = 4 * kParts;
   static constexpr int kMmaWarp = kSplitSoftmax ? kSoftWarps : 8;
   // one load warp takes K then V of each tile (a second warp for V measured
@@ -270,6 +275,7 @@ struct Bars {
   uint64_t k_full[kMaxKStages], k_empty[kMaxKStages], v_full[kMaxVStages], v_empty[kMaxVStages];
   uint64_t raw_full[kRawStages], raw_empty[kRawStages];
   uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2], done;
+  uint64_t pp_full[2][2];  // independent parts: P of part h in S buffer b written
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -386,6 +392,8 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       mbar_init(&B->s_full[s], 1);
       mbar_init(&B->s_empty[s], LY::kSoftWarps * 32);
       mbar_init(&B->p_full[s], LY::kSoftWarps * 32);
+      mbar_init(&B->pp_full[0][s], LY::kSoftWarps * 16);  // the 4 warps of a part
+      mbar_init(&B->pp_full[1][s], LY::kSoftWarps * 16);
       mbar_init(&B->pv_done[s], 1);
     }
     mbar_init(&B->done, 1);
@@ -459,7 +467,48 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       const uint32_t idesc_pv = idesc | (1u << 16);
       const uint32_t aQ = sbase + kQOff;
       bool ok = true;
-      for (int j = 0; j <= nkt && ok; ++j) {
+      if constexpr (LY::kIndep) {
+        // S(j) goes into TMEM buffer j % 2 once both parts' O += P V of tile
+        // j - 2 -- whose P was written over that buffer -- has completed.
+        // Then per tile: each part's O_h += P_h V_h (its 64 keys) as soon as
+        // that part's P is written.
+        auto issue_s = [&](int j) -> bool {
+          const int s = j & 1, sk = j % kKStages;
+          if (!wait_or_abort(&B->k_full[sk], (j / kKStages) & 1, B, p.dev_err)) return false;
+          if (j >= 2 && !wait_or_abort(&B->pv_done[s], ((j - 2) >> 1) & 1, B, p.dev_err))
+            return false;
+          tc_fence_after();
+          const uint32_t bK = sbase + kKOff + sk * kOpBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc_mma(tS + s * BN, smem_desc(aQ + off), smem_desc(bK + off), idesc, kk > 0);
+          }
+          tc_commit(&B->s_full[s]);
+          tc_commit(&B->k_empty[sk]);  // the K stage is free once S(j) is done
+          return true;
+        };
+        ok = issue_s(0) && (nkt < 2 || issue_s(1));
+        for (int jp = 0; jp < nkt && ok; ++jp) {
+          const int b = jp & 1, sv = jp % kVStages;
+          ok = wait_or_abort(&B->v_full[sv], (jp / kVStages) & 1, B, p.dev_err);
+          const uint32_t bV = sbase + kVOff + sv * kOpBytes;
+          for (int h = 0; h < 2 && ok; ++h) {
+            ok = wait_or_abort(&B->pp_full[h][b], (jp >> 1) & 1, B, p.dev_err);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // keys 64 h + 16 kk ..: two 8-row groups
+              tc_mma_ts(tO + h * 128, tS + b * BN + h * 64 + kk * 8,
+                        smem_desc(bV + (4 * h + kk) * 2048, 16384), idesc_pv, (jp > 0 || kk > 0));
+          }
+          if (!ok) break;
+          tc_commit(&B->pv_done[b]);
+          tc_commit(&B->v_empty[sv]);
+          if (jp + 2 < nkt) ok = issue_s(jp + 2);
+        }
+      }
+      for (int j = 0; j <= nkt && ok && !LY::kIndep; ++j) {
         if (j < nkt) {  // S(j) = Q K(j)^T into TMEM buffer j % 2
           const int s = j & 1, sk = j % kKStages;
           ok = wait_or_abort(&B->k_full[sk], (j / kKStages) & 1, B, p.dev_err);
@@ -721,6 +770,154 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
       for (int m = 0; m < 8; ++m) id_cur[m] = id_nxt[m];
       if (j + 2 < nkt) load_ids(j + 2, id_nxt);  // a whole tile ahead of its first use
     }
+    }
+  } else if constexpr (LY::kIndep) {
+    // ------------------------------ softmax, two independent parts per row
+    // Warps w and w + 4 share rows 32 (w % 4) .. + 31 (the TMEM lanes warp
+    // w % 4 may access); part hh takes keys 64 hh .. 64 hh + 63 of every tile
+    // with its own running max, sum and O accumulator O_hh (TMEM columns
+    // 256 + 128 hh), writes its P over the first half of its own S columns,
+    // and rescales only O_hh.  Nothing is exchanged per tile; at the end the
+    // two parts' (max, sum) meet in shared memory and each thread writes half
+    // of its row from both accumulators.
+    const int q4 = warp & 3, hh = warp >> 2;
+    const int r = q4 * 32 + lane;  // row = TMEM lane
+    const int i = i0 + r / G, g = r % G;
+    const bool row_valid = i < L;
+    const bool live = i0 + (q4 * 32) / G < L;  // see the split softmax below
+    const int lim = H + i;                      // last visible key
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tOh = tO + hh * 128 + lane_base;
+    const float sl = row_scale[r];  // > 0 exactly when the scale is
+    float m_used = -INFINITY, l = 0.f;
+    bool fail = false;  // warp-uniform
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j & 1;
+      fail = __any_sync(0xffffffffu, !wait_or_abort(&B->s_full[s], (j >> 1) & 1, B, p.dev_err));
+      if (fail) break;
+      tc_fence_after();
+      const int kbase = j * BN + hh * 64;  // first key of this part
+      const uint32_t tSrow = tS + lane_base + s * BN + hh * 64;
+      const bool full =
+          __all_sync(0xffffffffu, row_valid && kbase + 63 <= lim) && p.scale_log2 > 0.f;
+      float x[64];
+      float mx = -INFINITY;
+      if (live) {  // this part's scores and their max
+        tmem_ld32(tSrow, x);
+        tmem_ld32(tSrow + 32, x + 32);
+        tmem_wait_ld();
+        float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};  // 4 chains, not 1
+        if (full) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) m4[e & 3] = fmaxf(m4[e & 3], x[e]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const bool vis = !row_valid || (kbase + e <= lim);
+            m4[e & 3] = fmaxf(m4[e & 3], vis ? (row_valid ? x[e] * sl : 0.f) : -INFINITY);
+          }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+      }
+      // lazy rescale: only when this part's max grew by more than 2^8
+      const float m_new = fmaxf(m_used, mx);
+      const bool rescale = m_new > m_used + kRescaleLog2;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = exp2f(m_used - m_new);  // 0 on the first tile
+        l *= alpha;
+        m_used = m_new;
+      }
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};  // the row sum in 4 chains
+      uint32_t pk[32];
+      // a row that has seen no key yet exponentiates against 0 (P = 0, not NaN)
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      if (live) {
+        if (full) {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float a = fast_exp2(fmaf(x[e], sl, neg_m));
+            const float bb = fast_exp2(fmaf(x[e + 1], sl, neg_m));
+            r4[(e >> 1) & 3] += a + bb;
+            pk[e / 2] = pack2<false>(a, bb);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const int k0 = kbase + e;
+            const float v0 = row_valid ? (k0 <= lim ? x[e] * sl : -INFINITY) : 0.f;
+            const float v1 = row_valid ? (k0 + 1 <= lim ? x[e + 1] * sl : -INFINITY) : 0.f;
+            const float a = fast_exp2(v0 + neg_m), bb = fast_exp2(v1 + neg_m);
+            r4[(e >> 1) & 3] += a + bb;
+            pk[e / 2] = pack2<false>(a, bb);
+          }
+        }
+      }
+      l += (r4[0] + r4[1]) + (r4[2] + r4[3]);
+      // O_hh is rescaled (rarely) once O_hh += P V of tile j-1 has completed
+      if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
+        fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[(j - 1) & 1],
+                                                      ((j - 1) >> 1) & 1, B, p.dev_err));
+        if (fail) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float o[32];
+          tmem_ld32(tOh + cc * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tOh + cc * 32, o);
+        }
+        tmem_wait_st();
+      }
+      if (live) {
+        // the pair (key 2c, 2c+1) of this part in column c of its S columns
+        tc_fence_after();
+        tmem_st32(tSrow, reinterpret_cast<const float*>(pk));
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(&B->pp_full[hh][s]);
+    }
+    // epilogue: both parts' (max, sum) meet in shared memory once their last
+    // O += P V has completed; every softmax thread reaches the barrier once
+    if (!fail)
+      fail = __any_sync(0xffffffffu, !wait_or_abort(&B->pv_done[(nkt - 1) & 1],
+                                                    ((nkt - 1) >> 1) & 1, B, p.dev_err));
+    float2* red = reinterpret_cast<float2*>(smem + LY::kRedOff);  // [2][BM]
+    red[hh * BM + r] = make_float2(m_used, l);
+    if (!named_bar_or(2, LY::kSoftWarps * 32, fail)) {
+      tc_fence_after();
+      const float2 other = red[(hh ^ 1) * BM + r];
+      const float M = fmaxf(m_used, other.x);
+      const float w_me = m_used == -INFINITY ? 0.f : exp2f(m_used - M);
+      const float w_ot = other.x == -INFINITY ? 0.f : exp2f(other.x - M);
+      const float lt = w_me * l + w_ot * other.y;
+      const float inv = (lt > 0.f) ? p.out_mul / lt : 0.f;
+      const float w0 = (hh == 0 ? w_me : w_ot) * inv, w1 = (hh == 0 ? w_ot : w_me) * inv;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                           ((size_t)(q0 + (row_valid ? i : 0)) * p.n_q + (size_t)kvh * G + g) * D +
+                           hh * 64;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        float o0[32], o1[32];
+        tmem_ld32(tO + lane_base + hh * 64 + cc * 32, o0);
+        tmem_ld32(tO + 128 + lane_base + hh * 64 + cc * 32, o1);
+        tmem_wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack2<true>(o0[e] * w0 + o1[e] * w1, o0[e + 1] * w0 + o1[e + 1] * w1);
+            v.y = pack2<true>(o0[e + 2] * w0 + o1[e + 2] * w1, o0[e + 3] * w0 + o1[e + 3] * w1);
+            v.z = pack2<true>(o0[e + 4] * w0 + o1[e + 4] * w1, o0[e + 5] * w0 + o1[e + 5] * w1);
+            v.w = pack2<true>(o0[e + 6] * w0 + o1[e + 6] * w1, o0[e + 7] * w0 + o1[e + 7] * w1);
+            *reinterpret_cast<uint4*>(out + cc * 32 + e) = v;
+          }
+        }
+      }
     }
   } else if constexpr (LY::kSplitSoftmax) {
     // -------------------------------------- softmax, kParts warps per row
