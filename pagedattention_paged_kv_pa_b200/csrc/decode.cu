@@ -197,8 +197,13 @@ __device__ __forceinline__ void merge_and_store(float* mo, float* mm, float* ml,
 // (blockIdx.y = kv head x group quad); with cpc groups (cpc2 = cpc rounded up
 // to 1, 2 or 4) consumer warp w takes group w % cpc2 and every (4 / cpc2)-th
 // block, so one K/V stage serves all of the CTA's groups.
+// Registers: 96 with 16-bit caches (three CTAs per SM, a shared-memory
+// limit); 80 with fp8 caches, so that five CTAs fit an SM (96 allowed four):
+// the fp8 kernel is bound by its warps' per-block latency, and the fifth CTA
+// hides more of it than the few spilled registers cost (measured 403 against
+// 440 us on the mixed-step decode; 64 registers, six CTAs: 473 us).
 template <int D, bool FP8, bool Q_BF16, bool MQ>
-__global__ void __launch_bounds__(kThreads) decode_mma_kernel(
+__global__ void __launch_bounds__(kThreads) __maxnreg__(FP8 ? 80 : 96) decode_mma_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
     const DecodeParams p) {
   using L = MmaLayout<D, FP8>;
