@@ -277,6 +277,28 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_pool, const 
                             pa_dtype q_dtype, pa_dtype kv_dtype, float k_scale, float v_scale,
                             int32_t* dev_err, void* stream);
 
+/*
+ * pa_test_decode_timeout -- a test hook for the error path of the kernels'
+ * bounded waits; the pages have no counterpart to it.  It queues pa_decode
+ * (same arguments, q_dtype F16 or BF16) with every wait in the partition
+ * kernel giving up after wait_limit_us microseconds (1 .. 1,000,000; the
+ * library's own limit is 1 s) and with each CTA's producer warp leaving the
+ * shared-memory stage of its tile `skip_tile` unfilled, as if its load had
+ * never arrived.  The waits on that stage run out: the kernel sets
+ * PA_DEVERR_TIMEOUT in *dev_err, lets the loads it did issue land, and
+ * returns; the output is meaningless, the context stays usable, and the next
+ * call computes normally.  PA_ERR_INVALID_ARG for skip_tile < 0 or a limit
+ * out of range.
+ */
+pa_status pa_test_decode_timeout(void* out, const void* q, const void* k_pool,
+                                 const void* v_pool, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, int block_size,
+                                 int n_q_heads, int n_kv_heads, int head_dim, int num_seqs,
+                                 int max_blocks_per_seq, int num_blocks, pa_dtype q_dtype,
+                                 pa_dtype kv_dtype, float k_scale, float v_scale, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_err, void* stream,
+                                 int skip_tile, uint32_t wait_limit_us);
+
 /* ------------------------------------------------------------------------- */
 /* Chunked prefill                                                            */
 /* ------------------------------------------------------------------------- */

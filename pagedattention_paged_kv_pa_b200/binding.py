@@ -32,7 +32,7 @@ EXPORTS = (
     "pa_decode_multi", "pa_alloc_set_prefix_caching", "pa_alloc_admit",
     "pa_alloc_append_tokens", "pa_alloc_cached_list", "pa_alloc_num_cached",
     "pa_swap_blocks", "pa_decode_shared_prefix", "pa_prefix_groups",
-    "pa_prefill_workspace_size",
+    "pa_prefill_workspace_size", "pa_test_decode_timeout",
 )
 
 
@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
     L.pa_decode_reduce.argtypes = [P, P, I, I, I, I, I, I, F, P, Z, P]
     L.pa_decode_multi.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, F, F, P, Z,
                                   P, P]
+    L.pa_test_decode_timeout.argtypes = dec + [I, ctypes.c_uint32]
+    L.pa_test_decode_timeout.restype = I
     L.pa_decode_noalloc.argtypes = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, F, F, P, P]
     L.pa_decode_noalloc.restype = I
     L.pa_decode_noalloc_scratch_bytes.restype = Z
@@ -243,6 +245,21 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale, k_scale
     _check(lib.pa_decode(*_decode_args(out, q, k_pool, v_pool, block_tables, context_lens,
                                        scale, k_scale, v_scale, workspace, dev_err, stream)),
            "pa_decode")
+    return out
+
+
+def pa_test_decode_timeout(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                           skip_tile: int, wait_limit_us: int, k_scale=1.0, v_scale=1.0,
+                           workspace=None, dev_err=None, stream=None):
+    """Test hook: pa_decode with short bounded waits and one tile's stage left
+    unfilled in every CTA, so the waits run out (see include/pa.h)."""
+    if workspace is None:
+        workspace = alloc_decode_workspace(q, block_tables.shape[1])
+    _check(lib.pa_test_decode_timeout(*_decode_args(out, q, k_pool, v_pool, block_tables,
+                                                    context_lens, scale, k_scale, v_scale,
+                                                    workspace, dev_err, stream),
+                                      int(skip_tile), int(wait_limit_us)),
+           "pa_test_decode_timeout")
     return out
 
 

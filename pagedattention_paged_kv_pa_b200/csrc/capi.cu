@@ -196,7 +196,9 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
                                const int32_t* grp_members = nullptr,
                                const int32_t* grp_shared_blocks = nullptr,
                                const int32_t* seq_group = nullptr, int n_groups = 0,
-                               int grp_width = 0, bool tensor_core_multi = false) {
+                               int grp_width = 0, bool tensor_core_multi = false,
+                               unsigned long long wait_ns = pa::kWaitLimitNs,
+                               int skip_tile = -1) {
   DecodeShape s{n_q_heads, n_kv_heads, head_dim, num_seqs, max_blocks_per_seq, num_blocks,
                 pa::decode_num_parts(max_blocks_per_seq, pa::kPart16)};
   pa_status st = check_decode(s, block_size, q_dtype, kv_dtype);
@@ -251,6 +253,8 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
   p.grp_width = 0;
   p.n_groups = n_groups;
   p.n_seqs_all = num_seqs;
+  p.wait_ns = wait_ns;
+  p.skip_tile = skip_tile;
   CUtensorMap tmk, tmv;
   if (pa::decode_uses_tma(q_dtype, kv_dtype)) {
     if (!kv_pool_map(k_pool, num_blocks, n_kv_heads, head_dim, kv_dtype, &tmk) ||
@@ -357,6 +361,27 @@ pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_
   if (st != PA_OK) return st;
   return pa_decode_reduce(out, context_lens, n_q_heads, head_dim, num_seqs, max_blocks_per_seq,
                           q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_test_decode_timeout(void* out, const void* q, const void* k_pool,
+                                 const void* v_pool, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, int block_size,
+                                 int n_q_heads, int n_kv_heads, int head_dim, int num_seqs,
+                                 int max_blocks_per_seq, int num_blocks, pa_dtype q_dtype,
+                                 pa_dtype kv_dtype, float k_scale, float v_scale, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_err, void* stream,
+                                 int skip_tile, uint32_t wait_limit_us) {
+  if (skip_tile < 0 || wait_limit_us < 1 || wait_limit_us > 1000000) return PA_ERR_INVALID_ARG;
+  if (q_dtype == PA_F32) return PA_ERR_UNSUPPORTED;  // the TMA kernels only
+  pa_status st = decode_parts_impl(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                                   block_size, n_q_heads, n_kv_heads, head_dim, num_seqs, 1,
+                                   max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                                   v_scale, workspace, workspace_bytes, dev_err, stream, nullptr,
+                                   nullptr, nullptr, 0, 0, false,
+                                   (unsigned long long)wait_limit_us * 1000ull, skip_tile);
+  if (st != PA_OK) return st;
+  return decode_reduce_impl(out, context_lens, n_q_heads, head_dim, num_seqs, max_blocks_per_seq,
+                            q_dtype, kv_dtype, v_scale, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_decode_multi(void* out, const void* q, const void* k_pool, const void* v_pool,

@@ -319,14 +319,17 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(FP8 ? 80 : 96) decode_mm
       int issued = 0;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(&empty[s], ((j / kStages) - 1) & 1)) {
+        if (j >= kStages && !mbar_wait(&empty[s], ((j / kStages) - 1) & 1, p.wait_ns)) {
           flag_error(p.dev_err, PA_DEVERR_TIMEOUT);
           break;
         }
         const int id = ids[j];
         uint8_t* kt = smem + s * L::kStageBytes;
         uint8_t* vt = kt + L::kTileBytes;
-        if (id >= 0) {
+        if (j == p.skip_tile) {
+          // test hook (pa_test_decode_timeout): the stage is never filled, so
+          // the waits on it run out
+        } else if (id >= 0) {
           mbar_arrive_expect_tx(&full[s], 2 * L::kTileBytes);
           const int row = (id * p.n_kv + kvh) * 16;
           if (FP8 || D == 64) {
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(FP8 ? 80 : 96) decode_mm
       // Before the ring is reused as merge scratch, make sure no load issued
       // here is still landing (only matters if a consumer gave up early).
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        mbar_wait(&full[j % kStages], (j / kStages) & 1);
+        mbar_wait(&full[j % kStages], (j / kStages) & 1, p.wait_ns);
     }
   } else {
     // ------------------------------------------------------------ consumers
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(FP8 ? 80 : 96) decode_mm
 
     for (int j = active ? ph : nblk; j < nblk; j += wpg) {
       const int s = j % kStages;
-      if (!mbar_wait(&full[s], (j / kStages) & 1)) {
+      if (!mbar_wait(&full[s], (j / kStages) & 1, p.wait_ns)) {
         flag_error(p.dev_err, PA_DEVERR_TIMEOUT);
         break;
       }

@@ -12,12 +12,12 @@
 #include <cstdint>
 
 #include "../../include/pa.h"
+#include "pa_internal.h"
 
 namespace pa {
 
-// A bounded wait gives up after this long (the kernels' normal waits last
-// microseconds); the caller then records PA_DEVERR_TIMEOUT and winds down.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+// kWaitLimitNs (pa_internal.h): how long a bounded wait lasts before it gives
+// up; the caller then records PA_DEVERR_TIMEOUT and winds down.
 constexpr uint32_t kWaitLimitIters = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -68,13 +68,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false if the
-// wait gave up (time or iteration limit); it never spins forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// wait gave up (after limit_ns, or the iteration limit); it never spins
+// forever.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t i = 1; i < kWaitLimitIters; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 63) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
   }
   return false;
 }

@@ -11,6 +11,10 @@
 
 namespace pa {
 
+// A bounded wait inside a kernel gives up after this long (the kernels'
+// normal waits last microseconds) and flags PA_DEVERR_TIMEOUT.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+
 // Tokens per decode context partition: 1024 (64 blocks of 16) with 16-bit
 // and fp32 caches, 2048 with fp8 caches (about the same K/V bytes per CTA).
 // Longer partitions spread each CTA's fixed costs (block-table read, first
@@ -52,6 +56,10 @@ struct DecodeParams {
   int grp_width;
   int n_groups;     // for range checks of seq_group
   int n_seqs_all;   // for range checks of grp_members (num_seqs is the grid)
+  // bounded waits give up after wait_ns; skip_tile >= 0 (pa_test_decode_timeout
+  // only) makes each CTA's producer leave the stage of that tile unfilled
+  unsigned long long wait_ns;
+  int skip_tile;
 };
 
 struct ReduceParams {
