@@ -77,7 +77,7 @@ def _check(B, inp, qm, device, what):
 @pytest.mark.parametrize("q_dt,kv_dt", [(W.F16, W.F16), (W.BF16, W.BF16),
                                         (W.BF16, W.FP8_E4M3), (W.F16, W.FP8_E4M3)])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("q_len", [2, 5, 8])
 def test_dtype_group_qlen_grid(B, cuda_device, q_dt, kv_dt, d, G, q_len):
     n_kv = 2
