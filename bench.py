@@ -598,9 +598,9 @@ def extra_configs(dev, iters: int = 30):
                                           dev_err=err))
     res["spec_verify_bf16"] = hbm_entry(describe(spec, ctx, inp.num_blocks)
                                         + f"; {q_len} queries per sequence",
-                                        "pa_decode_multi: prefill_tc_kernel (bf16 tensor cores)",
+                                        "pa_decode_multi: mq_tc_kernel + mq_merge_kernel",
                                         ms, nbytes,
-                                        traffic=traffic_from_profile("spec_verify_bf16", "prefill"))
+                                        traffic=traffic_from_profile("spec_verify_bf16", "mq"))
     del inp, qm, out, ws
     # the mixed step's chunked prefill: widening pass + tensor-core kernel
     pspec = W.MIXED_PREFILL_FP8
@@ -796,6 +796,8 @@ def run_mixed(args, rank, world, local):
 
 DECODE_SOURCES = ("decode.cu", "pa_internal.h", "pa_device.cuh")
 PREFILL_SOURCES = ("prefill.cu", "pa_internal.h", "pa_device.cuh")
+MQ_SOURCES = ("decode_multi_tc.cu", "mq_tc.h", "tc_ops.cuh", "pa_internal.h", "pa_device.cuh")
+KERNEL_SOURCES = {"decode": DECODE_SOURCES, "prefill": PREFILL_SOURCES, "mq": MQ_SOURCES}
 
 
 def source_hash(files=DECODE_SOURCES):
@@ -813,12 +815,13 @@ def decode_source_hash():
 
 def traffic_from_profile(workload, kernel="decode"):
     """DRAM bytes per launch of the decode partition kernel (kernel="decode",
-    profiles/decode_traffic.txt) or of the tensor-core prefill kernel
-    (kernel="prefill", profiles/prefill_traffic.txt) from the committed ncu
+    profiles/decode_traffic.txt), of the tensor-core prefill kernel
+    (kernel="prefill", profiles/prefill_traffic.txt) or of the multi-query
+    kernel (kernel="mq", profiles/mq_traffic.txt) from the committed ncu
     summaries, if they were taken on the current kernel sources; None
     otherwise."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
-    files = DECODE_SOURCES if kernel == "decode" else PREFILL_SOURCES
+    files = KERNEL_SOURCES[kernel]
     try:
         rec = {}
         for line in open(path):
@@ -979,12 +982,13 @@ def run_spec_verify(args, rank, world, local):
                             "streams, double-buffered against the kernels"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": traffic_from_profile("spec_verify_bf16", "prefill"),
-                     "kernel": "pa_decode_multi: prefill_tc_kernel (bf16 tensor cores, one "
-                               "tile per sequence and kv head)",
+                     "traffic": traffic_from_profile("spec_verify_bf16", "mq"),
+                     "kernel": "pa_decode_multi: mq_tc_kernel (bf16 tensor cores, 64-row "
+                               "tiles, persistent CTAs with equal shares of the key tiles) + "
+                               "mq_merge_kernel (timed together)",
                      "kernel_avg_us": round(kern_ms * 1e3, 2),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
-        "gpu_launches": 2 * K,  # slot write + the tensor-core kernel
+        "gpu_launches": 3 * K,  # slot write + the multi-query kernel + its merge
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

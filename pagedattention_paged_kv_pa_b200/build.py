@@ -15,8 +15,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpa_b200.so")
 OBJDIR = os.path.join(ROOT, "_build", "obj")
 
-SOURCES = ["capi.cu", "decode.cu", "cache_ops.cu", "prefill.cu", "allocator.cpp",
-           "decode_noalloc.cu"]
+SOURCES = ["capi.cu", "decode.cu", "decode_multi_tc.cu", "cache_ops.cu", "prefill.cu",
+           "allocator.cpp", "decode_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE,

@@ -7,6 +7,7 @@
 #include <unordered_map>
 #include <vector>
 
+#include "mq_tc.h"
 #include "pa_internal.h"
 
 namespace {
@@ -117,6 +118,22 @@ bool kv_pool_map(const void* pool, int num_blocks, int n_kv, int d, pa_dtype dt,
   return get_map(pool, (uint64_t)num_blocks * n_kv * 16, d, es, box_x, 16, swz, m);
 }
 
+// Map over 16-bit queries [num_seqs x q_len][n_q][128] for the multi-query
+// tensor-core kernel: one box is the q_len x G rows of one kv head's query
+// heads, 64 columns wide (128-byte swizzle), landing as rows query x G + head.
+// Not cached: the query tensor usually changes from call to call.
+bool q_rows_map(const void* q, int rows, int n_q, int group, int q_len, CUtensorMap* m) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(n_q), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(n_q) * 256};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(q_len)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------ decode checks
 
 struct DecodeShape {
@@ -175,14 +192,16 @@ size_t pa_decode_workspace_size(int num_seqs, int n_q_heads, int head_dim, int m
 }
 
 // pa_decode_multi's step is the causal chunk of a sequence's q_len newest
-// queries over its cache, so for bf16 queries over a bf16 or fp8 cache with
-// head_dim 128 and group 1, 2, 4 or 8 it runs on the chunked-prefill
-// tensor-core kernel: one 128-row tile per (sequence, kv head) holds all
-// q_len x G (query, head) rows and reads each K/V tile once for them.
+// queries over its cache.  With head_dim 128 and group 1, 2, 4 or 8 it runs on
+// tensor cores, each K/V tile read once for all q_len x G (query, head) rows of
+// a kv head: 16-bit queries over a cache of the same type on the multi-query
+// kernel (64-row tiles, persistent CTAs with equal shares of the key tiles),
+// bf16 queries over an fp8 cache on the chunked-prefill kernel (one 128-row
+// tile per (sequence, kv head)).
 static bool multi_on_tensor_cores(int q_len, int head_dim, int group, pa_dtype q_dt,
                                   pa_dtype kv_dt) {
-  return q_len > 1 && head_dim == 128 && q_dt == PA_BF16 &&
-         (kv_dt == PA_BF16 || kv_dt == PA_FP8_E4M3) &&
+  const bool same16 = (q_dt == PA_BF16 || q_dt == PA_F16) && kv_dt == q_dt;
+  return q_len > 1 && head_dim == 128 && (same16 || (q_dt == PA_BF16 && kv_dt == PA_FP8_E4M3)) &&
          (group == 1 || group == 2 || group == 4 || group == 8);
 }
 
@@ -262,6 +281,28 @@ static pa_status decode_parts_impl(void* out, const void* q, const void* k_pool,
       return PA_ERR_CUDA;
   }
   const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (tensor_core_multi && kv_dtype == q_dtype) {
+    pa::MQParams mp;
+    mp.out = out;
+    mp.block_tables = block_tables;
+    mp.context_lens = context_lens;
+    mp.ws_o = p.ws_o;
+    mp.ws_ml = p.ws_ml;
+    mp.dev_err = dev_err;
+    mp.scale_log2 = p.scale_log2;
+    mp.n_q = n_q_heads;
+    mp.n_kv = n_kv_heads;
+    mp.group = p.group;
+    mp.q_len = q_len;
+    mp.num_seqs = num_seqs;
+    mp.max_blocks = max_blocks_per_seq;
+    mp.num_blocks = num_blocks;
+    mp.n_parts_max = s.n_parts;
+    CUtensorMap tmq;
+    if (!q_rows_map(q, num_seqs * q_len, n_q_heads, p.group, q_len, &tmq)) return PA_ERR_CUDA;
+    return cuda_status(pa::launch_mq_tc(mp, q_dtype == PA_BF16, k_pool, v_pool, &tmq, &tmk, &tmv,
+                                        n_grid > 1, cs));
+  }
   if (tensor_core_multi) {
     pa::PrefillParams pp;
     pp.out = out;
