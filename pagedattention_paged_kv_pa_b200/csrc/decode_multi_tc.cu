@@ -23,9 +23,9 @@
 //
 // Work split.  Persistent CTAs, one per SM.  The work is the (sequence, kv
 // head, 1024-token partition) units laid end to end in that order, measured
-// in key tiles; CTA c takes the units whose first tile lies in
-// [c T / C, (c + 1) T / C) (T tiles, C CTAs), so every CTA streams about the
-// same number of K/V bytes.  Consecutive partitions of one (sequence, kv
+// in key tiles plus a fixed cost per (sequence, kv head); CTA c takes the
+// units that start in [c T / C, (c + 1) T / C) (T in all, C CTAs), so every
+// CTA gets about the same time's worth of K/V streaming.  Consecutive partitions of one (sequence, kv
 // head) in a CTA form one segment, accumulated without a break.  A segment
 // that covers its whole (sequence, kv head) writes the normalised output
 // (and, if the sequence has more than one partition, marks the row's first
@@ -90,8 +90,8 @@ struct Bars {
   uint64_t k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS];
   uint64_t q_full[2], q_empty[2], s_full[2], s_empty[2], p_full, pv_done[2], o_free[2];
   uint64_t done;
-  long long gbase0;  // global tile index of (s0, kv head 0, tile 0)
-  long long gend;    // end of this CTA's share (global tile index)
+  long long gbase0;  // position of (s0, kv head 0) in the shares
+  long long gend;    // end of this CTA's share
   int s0, h0, p00;   // the first unit of the share (s0 >= num_seqs: none)
   uint32_t tmem_base;
   int abort_flag;
@@ -113,12 +113,20 @@ __device__ __forceinline__ int clamp_ctx(const MQParams& p, int s) {
   return c < 0 ? 0 : min(c, p.max_blocks * 16);
 }
 __device__ __forceinline__ int ctx_tiles(int ctx) { return (ctx + BN - 1) / BN; }
+// The shares are measured in key tiles plus kSegCost tiles' worth of time per
+// (sequence, kv head) -- a segment's fixed costs (its query load, its first
+// S, its epilogue after the last O += P V) -- so that a CTA whose share holds
+// many short sequences takes fewer tiles.  A (sequence, kv head) with nt key
+// tiles spans nt + kSegCost positions; its partition p starts at position
+// kSegCost + 8 p.
+constexpr int kSegCost = 3;
+__device__ __forceinline__ int seq_weight(int nt) { return nt > 0 ? nt + kSegCost : 0; }
 
 // A run of consecutive partitions p0 .. p1 (tiles t0 .. t1 - 1) of one
 // (sequence s, kv head h) inside this CTA's share.
 struct Seg {
   int s, h, p0, p1, t0, t1, ctx, nt, np;
-  long long gbase;  // global tile index of (s, kv head 0, tile 0)
+  long long gbase;  // position of (s, kv head 0) in the CTAs' shares
   bool whole;       // p0 .. p1 are all of (s, h)'s partitions
 };
 
@@ -132,13 +140,14 @@ __device__ bool seg_settle(const MQParams& p, Seg& g, long long gend) {
     g.p0 = 0;
     if (++g.h == p.n_kv) {
       g.h = 0;
-      g.gbase += (long long)p.n_kv * g.nt;
+      g.gbase += (long long)p.n_kv * seq_weight(g.nt);
       if (++g.s >= p.num_seqs) return false;
       g.ctx = clamp_ctx(p, g.s);
       g.nt = ctx_tiles(g.ctx);
     }
   }
-  const long long gsh = g.gbase + (long long)g.h * g.nt;
+  // position of (s, h)'s partition 0
+  const long long gsh = g.gbase + (long long)g.h * seq_weight(g.nt) + kSegCost;
   if (gsh + (long long)kPT * g.p0 >= gend) return false;
   const long long last = (gend - 1 - gsh) / kPT;  // last partition starting in the share
   g.p1 = (int)min((long long)(g.np - 1), last);
@@ -163,9 +172,9 @@ __device__ __forceinline__ bool seg_next(const MQParams& p, const Bars* B, Seg& 
   return seg_settle(p, g, B->gend);
 }
 
-// This CTA's share, found by one warp: T = n_kv x sum of the sequences' key
-// tiles; the share is [c T / C, (c + 1) T / C); its first unit is the first
-// partition whose first tile is at or after the share's start.
+// This CTA's share, found by one warp: T = n_kv x the sum of the sequences'
+// weights (seq_weight); the share is [c T / C, (c + 1) T / C); its first unit
+// is the first partition that starts at or after the share's start.
 __device__ void find_share(const MQParams& p, Bars* B, int lane) {
   const int S = p.num_seqs;
   long long part = 0;
@@ -173,7 +182,7 @@ __device__ void find_share(const MQParams& p, Bars* B, int lane) {
   for (int s = lane; s < S; s += 32) {
     const int c = __ldg(&p.context_lens[s]);
     over |= c > p.max_blocks * 16;
-    part += ctx_tiles(c < 0 ? 0 : min(c, p.max_blocks * 16));
+    part += seq_weight(ctx_tiles(c < 0 ? 0 : min(c, p.max_blocks * 16)));
   }
   if (blockIdx.x == 0 && __any_sync(0xffffffffu, over) && lane == 0)
     flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
@@ -190,7 +199,7 @@ __device__ void find_share(const MQParams& p, Bars* B, int lane) {
     long long acc = 0;  // global tile index of the chunk's first sequence
     for (int base = 0; base < S; base += 32) {
       const int s = base + lane;
-      const int n = s < S ? ctx_tiles(clamp_ctx(p, s)) : 0;
+      const int n = s < S ? seq_weight(ctx_tiles(clamp_ctx(p, s))) : 0;
       int incl = n;
 #pragma unroll
       for (int m = 1; m < 32; m <<= 1) {
@@ -206,7 +215,7 @@ __device__ void find_share(const MQParams& p, Bars* B, int lane) {
           const long long local = gbeg - gs;
           s0 = s;
           h0 = (int)(local / n);
-          p00 = (int)((local % n + kPT - 1) / kPT);
+          p00 = (int)((max(0LL, local % n - kSegCost) + kPT - 1) / kPT);
           gb = gs;
         }
         s0 = __shfl_sync(0xffffffffu, s0, src);
@@ -671,49 +680,56 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Combines the segments of the rows whose (sequence, kv head) was split
-// between CTAs: one warp per row, slots in increasing order, empty ones (max
-// -inf) skipped.  Rows of a sequence with one partition, and rows one CTA
-// finished (first slot's sum -1), were written by the attention kernel.
+// between CTAs.  A CTA takes 256 consecutive rows: one thread per row finds
+// the rows that need it (a sequence with more than one partition whose first
+// slot is not marked done), then one warp per such row merges its slots in
+// increasing order, empty ones (max -inf) skipped.  Rows of a sequence with
+// one partition, and rows one CTA finished, were written by the attention
+// kernel.
 template <typename OutT>
 __global__ void __launch_bounds__(256) mq_merge_kernel(const MQParams p) {
+  __shared__ int todo[256];
+  __shared__ int n_todo;
   pdl_wait();  // the attention kernel's results
-  const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (gw >= (long long)p.num_seqs * p.q_len * p.n_q) return;
-  const int s = (int)(gw / ((long long)p.q_len * p.n_q));
-  const int ctx = clamp_ctx(p, s);
-  const int np = (ctx + kPart16 - 1) / kPart16;
-  if (np <= 1) return;
-  const float2* ml = p.ws_ml + gw * p.n_parts_max;
-  if (ml[0].y == -1.f) return;
-  float M = -INFINITY;
-  for (int pp = lane; pp < np; pp += 32) M = fmaxf(M, ml[pp].x);
-  M = warp_max_xor(M, 1);
-  float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* wo = p.ws_o + gw * p.n_parts_max * D + lane * 4;
-  for (int pp = 0; pp < np; ++pp) {
-    const float2 v = ml[pp];
-    if (v.x == -INFINITY) continue;
-    const float w = exp2f(v.x - M);
-    L += w * v.y;
-    const float4 x = *reinterpret_cast<const float4*>(wo + (size_t)pp * D);
-    acc[0] += w * x.x;
-    acc[1] += w * x.y;
-    acc[2] += w * x.z;
-    acc[3] += w * x.w;
+  const long long rows = (long long)p.num_seqs * p.q_len * p.n_q;
+  const long long r0 = (long long)blockIdx.x * 256;
+  if (threadIdx.x == 0) n_todo = 0;
+  __syncthreads();
+  const long long r = r0 + threadIdx.x;
+  if (r < rows) {
+    const int s = (int)(r / ((long long)p.q_len * p.n_q));
+    const int np = (clamp_ctx(p, s) + kPart16 - 1) / kPart16;
+    if (np > 1 && p.ws_ml[r * p.n_parts_max].y != -1.f) todo[atomicAdd(&n_todo, 1)] = threadIdx.x;
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  OutT* out = reinterpret_cast<OutT*>(p.out) + gw * D + lane * 4;
-  if constexpr (std::is_same<OutT, __nv_bfloat16>::value) {
-    uint2 w;
-    w.x = pack2<true>(acc[0] * inv, acc[1] * inv);
-    w.y = pack2<true>(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out) = w;
-  } else {
-    uint2 w;
-    w.x = pack2<false>(acc[0] * inv, acc[1] * inv);
-    w.y = pack2<false>(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out) = w;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  for (int k = threadIdx.x >> 5; k < n_todo; k += 8) {
+    const long long gw = r0 + todo[k];
+    const int s = (int)(gw / ((long long)p.q_len * p.n_q));
+    const int np = (clamp_ctx(p, s) + kPart16 - 1) / kPart16;
+    const float2* ml = p.ws_ml + gw * p.n_parts_max;
+    float M = -INFINITY;
+    for (int pp = lane; pp < np; pp += 32) M = fmaxf(M, ml[pp].x);
+    M = warp_max_xor(M, 1);
+    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* wo = p.ws_o + gw * p.n_parts_max * D + lane * 4;
+    for (int pp = 0; pp < np; ++pp) {
+      const float2 v = ml[pp];
+      if (v.x == -INFINITY) continue;
+      const float w = exp2f(v.x - M);
+      L += w * v.y;
+      const float4 x = *reinterpret_cast<const float4*>(wo + (size_t)pp * D);
+      acc[0] += w * x.x;
+      acc[1] += w * x.y;
+      acc[2] += w * x.z;
+      acc[3] += w * x.w;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    constexpr bool kBf = std::is_same<OutT, __nv_bfloat16>::value;
+    uint2 o;
+    o.x = pack2<kBf>(acc[0] * inv, acc[1] * inv);
+    o.y = pack2<kBf>(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(reinterpret_cast<OutT*>(p.out) + gw * D + lane * 4) = o;
   }
 }
 
@@ -744,7 +760,7 @@ cudaError_t launch_t(const MQParams& p, const void* k_pool, const void* v_pool,
   if (e != cudaSuccess || !merge) return e;
   const long long rows = (long long)p.num_seqs * p.q_len * p.n_q;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((rows + 7) / 8));
+  cfg.gridDim = dim3((unsigned)((rows + 255) / 256));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
