@@ -27,12 +27,11 @@
 // units that start in [c T / C, (c + 1) T / C) (T in all, C CTAs), so every
 // CTA gets about the same time's worth of K/V streaming.  Consecutive partitions of one (sequence, kv
 // head) in a CTA form one segment, accumulated without a break.  A segment
-// that covers its whole (sequence, kv head) writes the normalised output
-// (and, if the sequence has more than one partition, marks the row's first
-// workspace slot "done" with a sum of -1); a segment of a (sequence, kv head)
-// split between CTAs writes its unnormalised output and (max, sum) to the
-// slot of its first partition and an empty state (max -inf) to its other
-// partitions' slots, and mq_merge_kernel combines them.  Sequences with no
+// that covers its whole (sequence, kv head) writes the normalised output; a
+// segment of a (sequence, kv head) split between CTAs writes its
+// unnormalised output and (max, sum) to the workspace slot of its first
+// partition and an empty state (max -inf) to its other partitions' slots, and
+// mq_merge_kernel combines them.  Sequences with no
 // context get all-zero rows.
 //
 // Roles: warps 0-3 softmax, warp 4 owns TMEM and issues the MMAs from one
@@ -172,60 +171,70 @@ __device__ __forceinline__ bool seg_next(const MQParams& p, const Bars* B, Seg& 
   return seg_settle(p, g, B->gend);
 }
 
-// This CTA's share, found by one warp: T = n_kv x the sum of the sequences'
-// weights (seq_weight); the share is [c T / C, (c + 1) T / C); its first unit
-// is the first partition that starts at or after the share's start.
-__device__ void find_share(const MQParams& p, Bars* B, int lane) {
-  const int S = p.num_seqs;
+// T = n_kv x the sum of the sequences' weights (seq_weight), by one warp;
+// flags contexts beyond the table (once, from CTA 0 when `report`).
+__device__ long long total_weight(const MQParams& p, int lane, bool report) {
   long long part = 0;
   bool over = false;
-  for (int s = lane; s < S; s += 32) {
+  for (int s = lane; s < p.num_seqs; s += 32) {
     const int c = __ldg(&p.context_lens[s]);
     over |= c > p.max_blocks * 16;
     part += seq_weight(ctx_tiles(c < 0 ? 0 : min(c, p.max_blocks * 16)));
   }
-  if (blockIdx.x == 0 && __any_sync(0xffffffffu, over) && lane == 0)
+  if (report && blockIdx.x == 0 && __any_sync(0xffffffffu, over) && lane == 0)
     flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-  const long long T = part * p.n_kv;
-  const long long C = gridDim.x, c = blockIdx.x;
-  // floor(c T / C) without overflow
-  const long long gbeg = (T / C) * c + (T % C) * c / C;
-  const long long gend = (T / C) * (c + 1) + (T % C) * (c + 1) / C;
-  int s0 = S, h0 = 0, p00 = 0;
-  long long gb = 0;
-  if (gbeg < gend) {
-    long long acc = 0;  // global tile index of the chunk's first sequence
-    for (int base = 0; base < S; base += 32) {
-      const int s = base + lane;
-      const int n = s < S ? seq_weight(ctx_tiles(clamp_ctx(p, s))) : 0;
-      int incl = n;
+  return part * p.n_kv;
+}
+// Start of share c of C: floor(c T / C) without overflow.
+__device__ __forceinline__ long long share_start(long long T, long long c, long long C) {
+  return (T / C) * c + (T % C) * c / C;
+}
+// The sequence s whose span of positions [gs, gs + n_kv w) contains X < T,
+// its position gs and its weight w, by one warp (the same values in every
+// lane); false when no sequence does.
+__device__ bool locate(const MQParams& p, long long X, int lane, int& s_out, long long& gs_out,
+                       int& w_out) {
+  long long acc = 0;  // position of the chunk's first sequence
+  for (int base = 0; base < p.num_seqs; base += 32) {
+    const int s = base + lane;
+    const int n = s < p.num_seqs ? seq_weight(ctx_tiles(clamp_ctx(p, s))) : 0;
+    int incl = n;
 #pragma unroll
-      for (int m = 1; m < 32; m <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, m);
-        if (lane >= m) incl += v;
-      }
-      const long long gs = acc + (long long)(incl - n) * p.n_kv;
-      const long long ge = acc + (long long)incl * p.n_kv;
-      const uint32_t hit = __ballot_sync(0xffffffffu, gs <= gbeg && gbeg < ge);
-      if (hit) {
-        const int src = __ffs(hit) - 1;
-        if (lane == src) {
-          const long long local = gbeg - gs;
-          s0 = s;
-          h0 = (int)(local / n);
-          p00 = (int)((max(0LL, local % n - kSegCost) + kPT - 1) / kPT);
-          gb = gs;
-        }
-        s0 = __shfl_sync(0xffffffffu, s0, src);
-        h0 = __shfl_sync(0xffffffffu, h0, src);
-        p00 = __shfl_sync(0xffffffffu, p00, src);
-        gb = __shfl_sync(0xffffffffu, gb, src);
-        break;
-      }
-      acc += (long long)__shfl_sync(0xffffffffu, incl, 31) * p.n_kv;
+    for (int m = 1; m < 32; m <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, m);
+      if (lane >= m) incl += v;
     }
+    const long long gs = acc + (long long)(incl - n) * p.n_kv;
+    const long long ge = acc + (long long)incl * p.n_kv;
+    const uint32_t hit = __ballot_sync(0xffffffffu, gs <= X && X < ge);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      s_out = __shfl_sync(0xffffffffu, s, src);
+      gs_out = __shfl_sync(0xffffffffu, gs, src);
+      w_out = __shfl_sync(0xffffffffu, n, src);
+      return true;
+    }
+    acc += (long long)__shfl_sync(0xffffffffu, incl, 31) * p.n_kv;
+  }
+  return false;
+}
+
+// This CTA's share [c T / C, (c + 1) T / C), found by one warp; its first
+// unit is the first partition that starts at or after the share's start.
+__device__ void find_share(const MQParams& p, Bars* B, int lane) {
+  const long long T = total_weight(p, lane, true);
+  const long long C = gridDim.x, c = blockIdx.x;
+  const long long gbeg = share_start(T, c, C), gend = share_start(T, c + 1, C);
+  int s0 = p.num_seqs, h0 = 0, p00 = 0, w = 0;
+  long long gb = 0;
+  if (gbeg < gend && locate(p, gbeg, lane, s0, gb, w)) {
+    const long long local = gbeg - gb;
+    h0 = (int)(local / w);
+    p00 = (int)((max(0LL, local % w - kSegCost) + kPT - 1) / kPT);
+  } else {
+    s0 = p.num_seqs;
   }
   if (lane == 0) {
     B->s0 = s0;
@@ -650,8 +659,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               out[(64 * (q >> 3) + 8 * (q & 7) + cpair) / 2] =
                   pack2<BF16>(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
             }
-            if (g.np > 1 && (lane & 3) == 0)
-              p.ws_ml[row * p.n_parts_max] = make_float2(m, -1.f);  // row done
           } else {
             float* wo = p.ws_o + (row * p.n_parts_max + g.p0) * D;
 #pragma unroll
@@ -679,34 +686,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Combines the segments of the rows whose (sequence, kv head) was split
-// between CTAs.  A CTA takes 256 consecutive rows: one thread per row finds
-// the rows that need it (a sequence with more than one partition whose first
-// slot is not marked done), then one warp per such row merges its slots in
-// increasing order, empty ones (max -inf) skipped.  Rows of a sequence with
-// one partition, and rows one CTA finished, were written by the attention
-// kernel.
+// Combines the segments of the (sequence, kv head) pairs split between CTAs.
+// Merge CTA c (the grid is the attention kernel's) looks at the boundary
+// between shares c and c + 1: if the (sequence, kv head) whose span holds
+// that boundary has partitions starting on both sides of it, and its first
+// partition lies in share c, this CTA merges its q_len x G rows -- so each
+// split pair is merged once, by the CTA of its first partition.  One warp per
+// row; the row's partition slots in increasing order, empty ones (max -inf)
+// skipped.  Every other row was written whole by the attention kernel.
 template <typename OutT>
 __global__ void __launch_bounds__(256) mq_merge_kernel(const MQParams p) {
-  __shared__ int todo[256];
-  __shared__ int n_todo;
-  pdl_wait();  // the attention kernel's results
-  const long long rows = (long long)p.num_seqs * p.q_len * p.n_q;
-  const long long r0 = (long long)blockIdx.x * 256;
-  if (threadIdx.x == 0) n_todo = 0;
-  __syncthreads();
-  const long long r = r0 + threadIdx.x;
-  if (r < rows) {
-    const int s = (int)(r / ((long long)p.q_len * p.n_q));
-    const int np = (clamp_ctx(p, s) + kPart16 - 1) / kPart16;
-    if (np > 1 && p.ws_ml[r * p.n_parts_max].y != -1.f) todo[atomicAdd(&n_todo, 1)] = threadIdx.x;
+  __shared__ int sh_s, sh_h, sh_np;
+  // finding the pair reads only the context lengths, so it overlaps the
+  // attention kernel (this grid is its programmatic dependent); the
+  // workspace is read after pdl_wait
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.group;
+  if (warp == 0) {
+    int s = -1, h = 0, np = 0;
+    const long long C = gridDim.x, c = blockIdx.x;
+    if (c + 1 < C) {
+      const long long T = total_weight(p, lane, false);
+      const long long X = share_start(T, c + 1, C);
+      int s0, w;
+      long long gs;
+      if (X < T && locate(p, X, lane, s0, gs, w)) {
+        const long long local = X - gs;
+        const int hh = (int)(local / w);
+        const long long r = local % w;  // X's offset in (s0, hh)'s span
+        const int npp = (w - kSegCost + kPT - 1) / kPT;
+        const int before = r <= kSegCost ? 0 : (int)((r - kSegCost + kPT - 1) / kPT);
+        if (before >= 1 && before < npp && gs + (long long)hh * w + kSegCost >= share_start(T, c, C)) {
+          s = s0;
+          h = hh;
+          np = npp;
+        }
+      }
+    }
+    if (lane == 0) {
+      sh_s = s;
+      sh_h = h;
+      sh_np = np;
+    }
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  for (int k = threadIdx.x >> 5; k < n_todo; k += 8) {
-    const long long gw = r0 + todo[k];
-    const int s = (int)(gw / ((long long)p.q_len * p.n_q));
-    const int np = (clamp_ctx(p, s) + kPart16 - 1) / kPart16;
+  pdl_wait();  // the attention kernel's results
+  if (sh_s < 0) return;
+  const int np = sh_np;
+  for (int k = warp; k < p.q_len * G; k += 8) {
+    const long long gw = ((long long)sh_s * p.q_len + k / G) * p.n_q + (long long)sh_h * G + k % G;
     const float2* ml = p.ws_ml + gw * p.n_parts_max;
     float M = -INFINITY;
     for (int pp = lane; pp < np; pp += 32) M = fmaxf(M, ml[pp].x);
@@ -716,13 +744,13 @@ __global__ void __launch_bounds__(256) mq_merge_kernel(const MQParams p) {
     for (int pp = 0; pp < np; ++pp) {
       const float2 v = ml[pp];
       if (v.x == -INFINITY) continue;
-      const float w = exp2f(v.x - M);
-      L += w * v.y;
+      const float wt = exp2f(v.x - M);
+      L += wt * v.y;
       const float4 x = *reinterpret_cast<const float4*>(wo + (size_t)pp * D);
-      acc[0] += w * x.x;
-      acc[1] += w * x.y;
-      acc[2] += w * x.z;
-      acc[3] += w * x.w;
+      acc[0] += wt * x.x;
+      acc[1] += wt * x.y;
+      acc[2] += wt * x.z;
+      acc[3] += wt * x.w;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     constexpr bool kBf = std::is_same<OutT, __nv_bfloat16>::value;
@@ -758,9 +786,8 @@ cudaError_t launch_t(const MQParams& p, const void* k_pool, const void* v_pool,
                                                                 *tmv);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !merge) return e;
-  const long long rows = (long long)p.num_seqs * p.q_len * p.n_q;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((rows + 255) / 256));
+  cfg.gridDim = dim3((unsigned)sm_count());  // one merge CTA per share boundary
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
