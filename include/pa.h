@@ -159,18 +159,28 @@ pa_status pa_decode_reduce(void* out, const int32_t* context_lens, int n_q_heads
  * A query whose position is negative (context_lens[s] < q_len - i) has no
  * keys and gets an all-zero row.  This is the causal chunk of
  * pa_prefill_paged with history context_lens[s] - q_len, and each K/V tile is
- * read once for all of a sequence's queries of a kv head: with bf16 queries,
- * head_dim 128, a bf16 or fp8 cache and group size 1, 2, 4 or 8 it runs on
- * pa_prefill_paged's tensor-core kernel (one 128-row tile holds the q_len x G
- * (query, head) rows of a kv head; no partitions, so the workspace is not
- * written), otherwise on decode's partition and merge kernels with up to 32
- * (query, head) pairs per tile pass.
+ * read once for all of a sequence's queries of a kv head.  Routes (head_dim
+ * 128, group size 1, 2, 4 or 8, q_len >= 2):
+ *  - bf16 or f16 queries over a cache of the same type: a multi-query
+ *    tensor-core kernel.  The q_len x G (query, head) rows of a kv head are
+ *    one 64-row tcgen05 tile; persistent CTAs, one per SM, take equal shares
+ *    of the work measured in 128-key tiles (plus a fixed cost per (sequence,
+ *    kv head)); a (sequence, kv head) whose keys are split between two CTAs
+ *    leaves its partial results in the workspace (the slots of its 1024-token
+ *    partitions) and a merge kernel combines them, all others are written
+ *    whole.  P enters O += P V as a bf16 value plus its bf16 residual (f16
+ *    queries: one f16 value).
+ *  - bf16 queries over an fp8 cache: pa_prefill_paged's tensor-core kernel
+ *    (one 128-row tile per (sequence, kv head); the workspace is not written).
+ *  - otherwise: decode's partition and merge kernels with up to 32 (query,
+ *    head) pairs per tile pass.
  *
  *   out, q       device [num_seqs][q_len][n_q_heads][head_dim], dtype q_dtype
  *   q_len        1 .. 8 (1 gives pa_decode's result)
  *   workspace    >= pa_decode_workspace_size(num_seqs, n_q_heads * q_len,
  *                head_dim, max_blocks_per_seq) bytes, 16-byte aligned (may be
- *                NULL when that size is 0)
+ *                NULL when that size is 0); scratch, contents on entry
+ *                ignored
  *   other arguments as pa_decode.
  *
  * Supported as pa_decode except q_dtype PA_F32 (PA_ERR_UNSUPPORTED);

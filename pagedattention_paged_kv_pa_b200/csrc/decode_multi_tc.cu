@@ -25,14 +25,14 @@
 // head, 1024-token partition) units laid end to end in that order, measured
 // in key tiles plus a fixed cost per (sequence, kv head); CTA c takes the
 // units that start in [c T / C, (c + 1) T / C) (T in all, C CTAs), so every
-// CTA gets about the same time's worth of K/V streaming.  Consecutive partitions of one (sequence, kv
-// head) in a CTA form one segment, accumulated without a break.  A segment
-// that covers its whole (sequence, kv head) writes the normalised output; a
-// segment of a (sequence, kv head) split between CTAs writes its
-// unnormalised output and (max, sum) to the workspace slot of its first
-// partition and an empty state (max -inf) to its other partitions' slots, and
-// mq_merge_kernel combines them.  Sequences with no
-// context get all-zero rows.
+// CTA gets about the same time's worth of K/V streaming.  Consecutive
+// partitions of one (sequence, kv head) in a CTA form one segment,
+// accumulated without a break.  A segment that covers its whole (sequence, kv
+// head) writes the normalised output; a segment of a (sequence, kv head)
+// split between CTAs writes its unnormalised output and (max, sum) to the
+// workspace slot of its first partition and an empty state (max -inf) to its
+// other partitions' slots, and mq_merge_kernel combines them.  Sequences with
+// no context get all-zero rows.
 //
 // Roles: warps 0-3 softmax, warp 4 owns TMEM and issues the MMAs from one
 // lane, warp 5 loads Q (one 3-D TMA box per 64-column half) and the K tiles
@@ -41,9 +41,8 @@
 // in, zeros after them, and zeros for blocks past the context or with an
 // out-of-range id, which the K warp flags).  Separate K and V warps keep a K
 // load from waiting for a V stage: K stages free up when S = Q K^T is done, V
-// stages only when O += P V is.  Every wait
-// is bounded; a CTA that gives up flags PA_DEVERR_TIMEOUT, drains its MMAs and
-// loads and frees TMEM.
+// stages only when O += P V is.  Every wait is bounded; a CTA that gives up
+// flags PA_DEVERR_TIMEOUT, drains its MMAs and loads and frees TMEM.
 #include <type_traits>
 
 #include "mq_tc.h"

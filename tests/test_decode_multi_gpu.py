@@ -6,9 +6,11 @@ keys 0 .. c - q_len + i: that is the oracle's causal chunk of q_len queries
 over a history of c - q_len ("LLM inference optimization", §五; "Daily AI,
 2026-07-31", 推測解碼).  When c < q_len the first q_len - c queries have no
 keys and must come back as zero rows; the others form a chunk of c queries
-over an empty history.  bf16 queries with head_dim 128 over a bf16 or fp8 cache
-(group 1, 2, 4 or 8) run on the chunked-prefill tensor-core kernel, the other
-cases on decode's partition and merge kernels; both are held to the oracle.
+over an empty history.  With head_dim 128 and group 1, 2, 4 or 8, bf16 or f16
+queries over a cache of the same type run on the multi-query tensor-core kernel
+(persistent CTAs with equal shares of the key tiles, split pairs merged), bf16
+queries over an fp8 cache on the chunked-prefill tensor-core kernel; the other
+cases on decode's partition and merge kernels.  All are held to the oracle.
 """
 import numpy as np
 import pytest
