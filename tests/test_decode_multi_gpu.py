@@ -206,3 +206,27 @@ def test_tensor_core_work_split(B, cuda_device, dt):
     a, _ = run_multi(B, inp, qm, cuda_device)
     b, _ = run_multi(B, inp, qm, cuda_device)
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("dt", [W.BF16, W.F16])
+def test_tensor_core_bad_table_entries(B, cuda_device, dt):
+    """On the multi-query kernel a block id outside the pool and a context
+    longer than its table are flagged (PA_DEVERR_BLOCK_ID), never read, and
+    leave the other sequences' rows as the oracle has them; the bad
+    sequences' rows stay finite."""
+    ctx = np.array([700, 1500, 300, 2100], np.int32)
+    spec = W.DecodeSpec("mq_bad", len(ctx), 16, 4, 128, dt, dt, "fixed", (ctx,), max_ctx=2304,
+                        pool_factor=1.2, seed=515)
+    inp = W.make_decode_inputs(spec, ctx=ctx)
+    inp.block_tables[1, 50] = inp.num_blocks + 7           # inside sequence 1's context
+    cl_bad = inp.context_lens.clone()
+    cl_bad[3] = inp.block_tables.shape[1] * 16 + 40        # beyond sequence 3's table
+    bad = W.DecodeInputs(inp.spec, inp.q, inp.k_pool, inp.v_pool, inp.block_tables, cl_bad,
+                         inp.scale, inp.k_scale, inp.v_scale)
+    qm = W.make_multi_queries(inp, 4, seed=516)
+    gpu, err = run_multi(B, bad, qm, cuda_device)
+    assert err & 1  # PA_DEVERR_BLOCK_ID
+    assert np.isfinite(gpu).all()
+    good = [0, 2]
+    ref = oracle_multi(P.subset_for_oracle(inp, good), qm[good].cpu())
+    P.assert_close(gpu[good], ref, dt, dt, "healthy sequences next to bad ones")
