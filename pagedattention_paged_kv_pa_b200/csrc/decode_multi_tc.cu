@@ -175,10 +175,19 @@ __device__ __forceinline__ bool seg_next(const MQParams& p, const Bars* B, Seg& 
 __device__ long long total_weight(const MQParams& p, int lane, bool report) {
   long long part = 0;
   bool over = false;
-  for (int s = lane; s < p.num_seqs; s += 32) {
-    const int c = __ldg(&p.context_lens[s]);
-    over |= c > p.max_blocks * 16;
-    part += seq_weight(ctx_tiles(c < 0 ? 0 : min(c, p.max_blocks * 16)));
+  // four independent loads in flight per lane
+  for (int s0 = lane; s0 < p.num_seqs; s0 += 128) {
+    int c[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0 + 32 * u;
+      c[u] = s < p.num_seqs ? __ldg(&p.context_lens[s]) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      over |= c[u] > p.max_blocks * 16;
+      part += seq_weight(ctx_tiles(c[u] < 0 ? 0 : min(c[u], p.max_blocks * 16)));
+    }
   }
   if (report && blockIdx.x == 0 && __any_sync(0xffffffffu, over) && lane == 0)
     flag_error(p.dev_err, PA_DEVERR_BLOCK_ID);
@@ -196,9 +205,14 @@ __device__ __forceinline__ long long share_start(long long T, long long c, long 
 __device__ bool locate(const MQParams& p, long long X, int lane, int& s_out, long long& gs_out,
                        int& w_out) {
   long long acc = 0;  // position of the chunk's first sequence
+  // the next chunk's context length is loaded while this one is scanned
+  int c_next = lane < p.num_seqs ? __ldg(&p.context_lens[lane]) : 0;
   for (int base = 0; base < p.num_seqs; base += 32) {
     const int s = base + lane;
-    const int n = s < p.num_seqs ? seq_weight(ctx_tiles(clamp_ctx(p, s))) : 0;
+    const int c = c_next;
+    c_next = s + 32 < p.num_seqs ? __ldg(&p.context_lens[s + 32]) : 0;
+    const int cc = c < 0 ? 0 : min(c, p.max_blocks * 16);
+    const int n = s < p.num_seqs ? seq_weight(ctx_tiles(cc)) : 0;
     int incl = n;
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {

@@ -230,3 +230,17 @@ def test_tensor_core_bad_table_entries(B, cuda_device, dt):
     good = [0, 2]
     ref = oracle_multi(P.subset_for_oracle(inp, good), qm[good].cpu())
     P.assert_close(gpu[good], ref, dt, dt, "healthy sequences next to bad ones")
+
+
+def test_tensor_core_many_sequences(B, cuda_device):
+    """A batch of 1,000 short sequences (not a multiple of the 32 or 128 the
+    kernel's share search takes at a time; a tenth of them empty) on the
+    multi-query kernel: every row against the oracle."""
+    rng = np.random.default_rng(1000)
+    ctx = rng.integers(1, 600, size=1000).astype(np.int32)
+    ctx[rng.choice(1000, size=100, replace=False)] = 0
+    spec = W.DecodeSpec("mq_many", len(ctx), 8, 2, 128, W.BF16, W.BF16, "fixed", (ctx,),
+                        max_ctx=640, pool_factor=1.1, seed=1001)
+    inp = W.make_decode_inputs(spec, ctx=ctx)
+    qm = W.make_multi_queries(inp, 3, seed=1002)
+    _check(B, inp, qm, cuda_device, "1,000 sequences")
