@@ -5,7 +5,8 @@ bf16 queries, keys and values far outside f16's range (|x| of 1e5 and more)
 or deep in its subnormal range (1e-6) must give the oracle's result on every
 path: chunked prefill with a bf16 cache (bf16 tensor-core operands) and with
 an fp8 cache (E4M3 widened to f16, each bf16 query row scaled into f16's range
-by a power of two), and decode with either cache.
+by a power of two), decode with either cache, and multi-query decode (its
+tcgen05 kernel with a bf16 cache, the prefill kernel with an fp8 cache).
 
 Three kinds of input, all on top of the usual seeded N(0,1) draws:
   * powers of two that cancel in the scores (q x 2^-a with k x 2^a, or with
@@ -250,3 +251,52 @@ def test_decode_multi_fp8_query_rows_far_from_f16_range(B, cuda_device):
         assert err == 0
         P.assert_close(gpu, oracle_multi(sub, q), W.BF16, W.FP8_E4M3,
                        f"multi-query decode fp8, q x 2^{-e}")
+
+
+# --------------------------------------------- multi-query (tcgen05 kernel)
+
+def _multi_check(B, inp, qm, dev, what, out_scale=1.0):
+    from tests.test_decode_multi_gpu import oracle_multi, run_multi
+    gpu, err = run_multi(B, inp, qm, dev)
+    assert err == 0
+    ref = oracle_multi(inp, qm)
+    P.assert_close(gpu * out_scale, ref * out_scale, W.BF16, W.BF16, what)
+
+
+def test_decode_multi_bf16_keys_beyond_f16_range(B, cuda_device):
+    inp = _decode_inputs(W.BF16, 421)
+    qm = W.make_multi_queries(inp, 3, seed=10)
+    inp = dataclasses.replace(inp, k_pool=_times(inp.k_pool, 2.0 ** 15))
+    _multi_check(B, inp, _times(qm, 2.0 ** -15), cuda_device,
+                 "multi-query decode bf16, q x 2^-15, K x 2^15")
+
+
+@pytest.mark.parametrize("e", [17, -20])
+def test_decode_multi_bf16_values_scaled(B, cuda_device, e):
+    inp = _decode_inputs(W.BF16, 422)
+    qm = W.make_multi_queries(inp, 3, seed=11)
+    inp = dataclasses.replace(inp, v_pool=_times(inp.v_pool, 2.0 ** e))
+    _multi_check(B, inp, qm, cuda_device, f"multi-query decode bf16, V x 2^{e}",
+                 out_scale=2.0 ** -e)
+
+
+def test_decode_multi_bf16_planted_queries_and_keys(B, cuda_device):
+    inp = _decode_inputs(W.BF16, 423)
+    qm = W.make_multi_queries(inp, 3, seed=12)
+    qm = _plant(qm, Q_PLANT_DIMS, 0.05, 13, zero_dims=K_PLANT_DIMS)
+    inp = dataclasses.replace(inp, k_pool=_plant(inp.k_pool, K_PLANT_DIMS, 0.05, 14,
+                                                 zero_dims=Q_PLANT_DIMS))
+    _multi_check(B, inp, qm, cuda_device, "multi-query decode bf16, planted queries and keys")
+
+
+def test_decode_multi_bf16_planted_values(B, cuda_device):
+    from tests.test_decode_multi_gpu import oracle_multi, run_multi
+    inp = _decode_inputs(W.BF16, 424)
+    qm = W.make_multi_queries(inp, 3, seed=15)
+    inp = dataclasses.replace(inp, v_pool=_plant(inp.v_pool, range(128), 0.002, 16))
+    gpu, err = run_multi(B, inp, qm, cuda_device)
+    assert err == 0
+    ref = oracle_multi(inp, qm)
+    assert np.abs(ref).max() > 1e4
+    mag = oracle_multi(dataclasses.replace(inp, v_pool=inp.v_pool.abs()), qm)
+    _assert_close_mag(gpu, ref, mag, "multi-query decode bf16, planted values")
